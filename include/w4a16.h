@@ -1,0 +1,167 @@
+/*
+ * w4a16.h — C ABI of the B200 (sm_100a) weight-only int4 linear layer.
+ *
+ * The layer (vLLM PR #37352 analysis page, "[vllm] AMD ROCm을 위한 Triton 기반
+ * W4A16 커널 도입", section "코드 분석 1. Triton 기반 GEMM 커널 구현 및 검증"):
+ *
+ *     out[M, N] = fp16( fp32(A[M, K]) @ W[K, N] ),   W[k, n] = (q[k, n] - z[k/G, n]) * s[k/G, n]
+ *
+ * with q the unsigned int4 weight, s the fp16 group scale, z the int4 zero point
+ * (packed per group, or the constant zp_bias for symmetric quantisation) and an
+ * fp32 accumulator.
+ *
+ * Data layouts (all dense, row-major, no padding between rows):
+ *   A        fp16  [M, K]
+ *   b_packed int32 [K, N/8]    word (k, c), nibble j (bits 4j..4j+3) = q[k, 8c + j]
+ *   scales   fp16  [K/G, N]
+ *   qzeros   int32 [K/G, N/8]  word (g, c), nibble j = z[g, 8c + j]
+ *   out      fp16  [M, N]
+ *   ckpt     int32 [N, K/8]    checkpoint layout: word (n, c), nibble j = q[8c + j, n]
+ * Nibbles are unsigned (0..15). The nibble order inside a word is not printed on
+ * the page; the order above (element 8c + j in nibble j) is the reading taken.
+ *
+ * Common rules for every entry point:
+ *   - Every pointer argument is a DEVICE pointer (CUDA global memory) unless the
+ *     comment says otherwise. The caller owns every buffer; the library never
+ *     allocates, frees or retains a pointer after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Work is enqueued on it asynchronously; no entry point
+ *     synchronises the device or the stream, except w4a16_workspace_status.
+ *   - Arguments are checked on the host before any launch. A failed check
+ *     returns W4A16_ERR_INVALID_ARG (or W4A16_ERR_UNSUPPORTED) and launches
+ *     nothing. A launch failure returns W4A16_ERR_CUDA; the CUDA error text is
+ *     then available from w4a16_last_error() on the calling thread.
+ *   - The library is thread-safe. Its only global state is a per-device cache
+ *     of device attributes (SM count).
+ *   - The CUDA path is the only path: there is no CPU fallback.
+ */
+#ifndef W4A16_H_
+#define W4A16_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W4A16_API __attribute__((visibility("default")))
+#else
+#define W4A16_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4A16_OK = 0,
+    W4A16_ERR_INVALID_ARG = 1,   /* an argument failed a host-side check; nothing launched */
+    W4A16_ERR_UNSUPPORTED = 2,   /* valid arguments this build cannot run (e.g. not an sm_100 device) */
+    W4A16_ERR_CUDA = 3,          /* a CUDA call or launch failed; see w4a16_last_error() */
+    W4A16_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (read via w4a16_workspace_status) */
+} w4a16_status;
+
+/*
+ * w4a16_repack — checkpoint layout [N, K/8] to kernel layout [K, N/8], bit-exact.
+ *
+ * Cited operation: section "2. 가중치 레이아웃 재포장 (Weight Repacking)" of the
+ * PR #37352 analysis page: the compressed-tensors checkpoint weight [N, K//8]
+ * becomes the kernel's [K, N//8] after loading.
+ *
+ *   ckpt_nk8  const int32 [N, K/8], device, 4-byte aligned; read only.
+ *   out_kn8   int32 [K, N/8], device, 4-byte aligned; fully overwritten.
+ *             Must not overlap ckpt_nk8.
+ *   N, K      N >= 8, K >= 8, N % 8 == 0, K % 8 == 0.
+ * Errors: INVALID_ARG for a NULL pointer, a size rule broken, misalignment or
+ * overlapping buffers; CUDA for a launch failure.
+ */
+W4A16_API w4a16_status w4a16_repack(const void* ckpt_nk8, void* out_kn8, int64_t N, int64_t K, void* stream);
+
+/*
+ * w4a16_gemm_workspace_bytes — bytes of device workspace w4a16_gemm needs for
+ * this shape on the current device (0 when the shape needs none). Returns 0 for
+ * shapes w4a16_gemm would reject. The value depends on the current device's SM
+ * count; query it with the device current on which the GEMM will run.
+ */
+W4A16_API size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size);
+
+/*
+ * w4a16_gemm — out = fp16(fp32(A) @ ((q - z) * s)).
+ *
+ * Cited operation: the `_w4a16_reference` excerpt and the
+ * `triton_w4a16_gemm(a, b_q, scales, qzeros, group_size, zp_bias)` call in
+ * section "코드 분석 1" of the PR #37352 analysis page; the contiguity and
+ * N % 8 checks follow section "3. 엄격한 데이터 정렬 및 연속성 보장".
+ *
+ *   a         const fp16 [M, K], device, 2-byte aligned.
+ *   b_packed  const int32 [K, N/8], device, 4-byte aligned.
+ *   scales    const fp16 [K/G, N], device, 2-byte aligned.
+ *   qzeros    const int32 [K/G, N/8], device, 4-byte aligned; or NULL for the
+ *             symmetric form, where every zero point is zp_bias. When qzeros is
+ *             given, zp_bias is ignored.
+ *   M, N, K   M >= 1, N >= 8, K >= group_size; N % 8 == 0; K % group_size == 0.
+ *             M <= 8 runs the CUDA-core GEMV; M >= 9 the tensor-core GEMM.
+ *   group_size G: G >= 16 and G % 16 == 0.
+ *   zp_bias   0..15 when qzeros is NULL.
+ *   out       fp16 [M, N], device, 2-byte aligned; fully overwritten; must not
+ *             overlap any input.
+ *   workspace device buffer of at least w4a16_gemm_workspace_bytes(M, N, K, G)
+ *             bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE. Every
+ *             call leaves it as it found it (its counters are reset by the
+ *             kernels), so one zero-fill serves any number of calls. Calls that
+ *             share a workspace must be ordered (same stream, or events).
+ *             May be NULL when the query returned 0.
+ *   stream    cudaStream_t as void*.
+ * Accumulation is fp32; the group scale is applied in fp32 after each group's
+ * exact (q - z) * a partial sums; the result is rounded to fp16 to nearest even.
+ * Repeated calls with the same inputs give bit-identical outputs (fixed
+ * reduction order, no floating-point atomics).
+ * Errors: INVALID_ARG for a NULL required pointer, a size rule broken, a short
+ * or misaligned workspace or misaligned data; UNSUPPORTED when the current
+ * device is not sm_100; CUDA for a launch failure.
+ */
+W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const void* scales, const void* qzeros,
+                        int64_t M, int64_t N, int64_t K, int32_t group_size, int32_t zp_bias,
+                        void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Kernel selection for tests and measurement. kernel: W4A16_KERNEL_AUTO uses
+ * the same table as w4a16_gemm; GEMV forces the CUDA-core GEMV (any M; M > 8
+ * runs it once per 8-row block of A); TC forces the tensor-core GEMM.
+ * split_k: 0 = automatic, else the number of K slices (1..256) the GEMV splits
+ * its work into (ignored by the tensor-core GEMM).
+ */
+enum { W4A16_KERNEL_AUTO = 0, W4A16_KERNEL_GEMV = 1, W4A16_KERNEL_TC = 2 };
+typedef struct {
+    int32_t kernel;
+    int32_t split_k;
+} w4a16_gemm_options;
+
+/* Workspace bytes for w4a16_gemm_ex with these options (NULL opts = automatic). */
+W4A16_API size_t w4a16_gemm_ex_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size,
+                                     const w4a16_gemm_options* opts);
+
+/* w4a16_gemm with explicit kernel options (NULL opts = w4a16_gemm). Same contract. */
+W4A16_API w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scales, const void* qzeros,
+                           int64_t M, int64_t N, int64_t K, int32_t group_size, int32_t zp_bias,
+                           void* out, void* workspace, size_t workspace_bytes, void* stream,
+                           const w4a16_gemm_options* opts);
+
+/*
+ * w4a16_workspace_status — read the device status word kept at the start of a
+ * GEMM workspace into *status (a w4a16_status value; W4A16_OK unless a bounded
+ * device-side wait gave up). Synchronises `stream`. The word is sticky: pass
+ * clear != 0 to reset it to W4A16_OK after reading.
+ * Errors: INVALID_ARG for NULL pointers; CUDA for a failed copy.
+ */
+W4A16_API w4a16_status w4a16_workspace_status(void* workspace, int32_t clear, int32_t* status, void* stream);
+
+/* Static description of a status code. Never NULL. */
+W4A16_API const char* w4a16_status_string(w4a16_status s);
+
+/* Text of the last error on the calling thread ("" when none). Never NULL. */
+W4A16_API const char* w4a16_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H_ */

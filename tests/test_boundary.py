@@ -1,0 +1,125 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every symbol
+include/w4a16.h declares, and rejects bad arguments on the host with a status
+code before any CUDA call (nothing is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_only_int4_08_b200 as w
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names |= set(re.findall(r"W4A16_API\s+[\w\s\*]+?\b(w4a16_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ("w4a16_repack", "w4a16_gemm", "w4a16_gemm_workspace_bytes", "w4a16_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert names
+    for n in names:
+        assert hasattr(w.lib, n), n
+    assert set(w.EXPORTED) == names
+
+
+def test_status_strings():
+    for code, text in [(0, "ok"), (1, "invalid argument"), (2, "unsupported"), (3, "CUDA error"),
+                       (4, "device wait timed out"), (99, "unknown status")]:
+        assert w.w4a16_status_string(code) == text
+
+
+P = ctypes.c_void_p
+GOOD = P(0x10000)        # well-aligned dummy addresses: never dereferenced on failure
+GOOD2 = P(0x20000000)
+GOOD3 = P(0x40000000)
+OUT = P(0x60000000)
+
+
+def gemm(a=GOOD, b=GOOD2, s=GOOD3, z=None, M=1, N=64, K=256, G=128, zp=8, out=OUT, ws=None, wsb=0):
+    return w.lib.w4a16_gemm(a, b, s, z, M, N, K, G, zp, out, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(a=None), "NULL pointer"),
+    (dict(b=None), "NULL pointer"),
+    (dict(s=None), "NULL pointer"),
+    (dict(out=None), "NULL pointer"),
+    (dict(M=0), "M must be"),
+    (dict(M=-3), "M must be"),
+    (dict(N=60), "N must be"),
+    (dict(N=0), "N must be"),
+    (dict(K=200), "K must be"),
+    (dict(K=64), "K must be"),
+    (dict(G=100), "group_size"),
+    (dict(G=8, K=64), "group_size"),
+    (dict(G=0), "group_size"),
+    (dict(zp=16), "zp_bias"),
+    (dict(zp=-1), "zp_bias"),
+    (dict(a=P(0x10001)), "aligned"),
+    (dict(b=P(0x20000002)), "aligned"),
+    (dict(z=P(0x30000001)), "aligned"),
+    (dict(out=P(0x10000)), "overlaps"),
+    (dict(M=1 << 31), "too large"),
+])
+def test_gemm_rejects_bad_arguments_on_host(kw, why):
+    rc = gemm(**kw)
+    assert rc == w.W4A16_ERR_INVALID_ARG
+    assert why in w.lib.w4a16_last_error().decode()
+
+
+def test_zp_bias_not_checked_when_zeros_given():
+    # with qzeros the zp_bias is ignored; the call then fails later (no GPU here), not on zp_bias
+    gemm(z=P(0x30000000), zp=99)
+    assert "zp_bias" not in w.lib.w4a16_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(c=None), "NULL"), (dict(o=None), "NULL"),
+    (dict(N=12), "N must be"), (dict(K=4), "K must be"), (dict(N=0), "N must be"),
+    (dict(c=P(0x1002)), "aligned"), (dict(o=P(0x1000), c=P(0x1000)), "overlap"),
+])
+def test_repack_rejects_bad_arguments_on_host(kw, why):
+    c = kw.get("c", P(0x1000))
+    o = kw.get("o", P(0x80000000))
+    rc = w.lib.w4a16_repack(c, o, kw.get("N", 64), kw.get("K", 64), None)
+    assert rc == w.W4A16_ERR_INVALID_ARG
+    assert why in w.lib.w4a16_last_error().decode()
+
+
+def test_options_are_checked():
+    o = w.W4A16Options(7, 0)
+    rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
+    assert rc == w.W4A16_ERR_INVALID_ARG
+    o = w.W4A16Options(1, 999)
+    rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
+    assert rc == w.W4A16_ERR_INVALID_ARG
+
+
+def test_workspace_query_rejects_bad_shapes():
+    assert w.lib.w4a16_gemm_workspace_bytes(1, 60, 256, 128) == 0
+    assert w.lib.w4a16_gemm_workspace_bytes(0, 64, 256, 128) == 0
+
+
+def test_workspace_status_null_checks():
+    v = ctypes.c_int32()
+    assert w.lib.w4a16_workspace_status(None, 0, ctypes.byref(v), None) == w.W4A16_ERR_INVALID_ARG
+
+
+def test_python_binding_requires_cuda_tensors():
+    import torch
+    a = torch.zeros(1, 256, dtype=torch.float16)
+    with pytest.raises(TypeError):
+        w.w4a16_gemm(a, torch.zeros(256, 8, dtype=torch.int32), torch.zeros(2, 64, dtype=torch.float16), None, 128)

@@ -1,0 +1,158 @@
+"""B200 (sm_100a) weight-only int4 linear layer: thin Python binding of libw4a16.so.
+
+The functions here only marshal arguments to the C ABI declared in
+include/w4a16.h (same names); every step of the computation runs in the
+library's CUDA kernels. PyTorch supplies device memory and the current stream.
+There is no CPU fallback: importing this package fails if the library is not
+built (``python -m weight_only_int4_08_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libw4a16.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m weight_only_int4_08_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+W4A16_OK, W4A16_ERR_INVALID_ARG, W4A16_ERR_UNSUPPORTED, W4A16_ERR_CUDA, W4A16_ERR_TIMEOUT = range(5)
+KERNEL_AUTO, KERNEL_GEMV, KERNEL_TC = 0, 1, 2
+
+
+class W4A16Options(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("split_k", ctypes.c_int32)]
+
+
+_p, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+lib.w4a16_repack.argtypes = [_p, _p, _i64, _i64, _p]
+lib.w4a16_repack.restype = ctypes.c_int
+lib.w4a16_gemm_workspace_bytes.argtypes = [_i64, _i64, _i64, _i32]
+lib.w4a16_gemm_workspace_bytes.restype = _sz
+lib.w4a16_gemm_ex_workspace_bytes.argtypes = [_i64, _i64, _i64, _i32, ctypes.POINTER(W4A16Options)]
+lib.w4a16_gemm_ex_workspace_bytes.restype = _sz
+lib.w4a16_gemm.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _i32, _p, _p, _sz, _p]
+lib.w4a16_gemm.restype = ctypes.c_int
+lib.w4a16_gemm_ex.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _i32, _p, _p, _sz, _p,
+                              ctypes.POINTER(W4A16Options)]
+lib.w4a16_gemm_ex.restype = ctypes.c_int
+lib.w4a16_workspace_status.argtypes = [_p, _i32, ctypes.POINTER(ctypes.c_int32), _p]
+lib.w4a16_workspace_status.restype = ctypes.c_int
+lib.w4a16_status_string.argtypes = [ctypes.c_int]
+lib.w4a16_status_string.restype = ctypes.c_char_p
+lib.w4a16_last_error.argtypes = []
+lib.w4a16_last_error.restype = ctypes.c_char_p
+
+EXPORTED = ("w4a16_repack", "w4a16_gemm_workspace_bytes", "w4a16_gemm", "w4a16_gemm_ex_workspace_bytes",
+            "w4a16_gemm_ex", "w4a16_workspace_status", "w4a16_status_string", "w4a16_last_error")
+
+
+class W4A16Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.w4a16_last_error().decode() or lib.w4a16_status_string(status).decode()
+        super().__init__(f"{where}: {lib.w4a16_status_string(status).decode()} ({msg})")
+
+
+def _check(rc: int, where: str):
+    if rc != W4A16_OK:
+        raise W4A16Error(rc, where)
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, name, dtype):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtype:
+        raise TypeError(f"{name} must have dtype in {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _opts(kernel, split_k):
+    if kernel is None and not split_k:
+        return None
+    return ctypes.byref(W4A16Options(int(kernel or KERNEL_AUTO), int(split_k or 0)))
+
+
+def w4a16_status_string(status: int) -> str:
+    return lib.w4a16_status_string(int(status)).decode()
+
+
+def w4a16_gemm_workspace_bytes(M: int, N: int, K: int, group_size: int, kernel=None, split_k: int = 0) -> int:
+    o = _opts(kernel, split_k)
+    if o is None:
+        return int(lib.w4a16_gemm_workspace_bytes(M, N, K, group_size))
+    return int(lib.w4a16_gemm_ex_workspace_bytes(M, N, K, group_size, o))
+
+
+def alloc_workspace(M: int, N: int, K: int, group_size: int, device=None, kernel=None, split_k: int = 0):
+    """Zero-filled workspace for w4a16_gemm (reusable by every later call of that shape)."""
+    n = w4a16_gemm_workspace_bytes(M, N, K, group_size, kernel, split_k)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def w4a16_repack(ckpt_nk8: torch.Tensor, N: int, K: int, out: torch.Tensor | None = None, stream=None):
+    """Checkpoint [N, K/8] int32 -> kernel [K, N/8] int32 (bit-exact), on the GPU."""
+    pc = _dev(ckpt_nk8, "ckpt_nk8", (torch.int32, torch.uint32))
+    if ckpt_nk8.numel() != N * K // 8:
+        raise ValueError("ckpt_nk8 must have N*K/8 elements")
+    if out is None:
+        out = torch.empty((K, N // 8), dtype=torch.int32, device=ckpt_nk8.device)
+    po = _dev(out, "out", (torch.int32, torch.uint32))
+    if out.numel() != N * K // 8:
+        raise ValueError("out must have N*K/8 elements")
+    _check(lib.w4a16_repack(pc, po, N, K, _stream_ptr(stream)), "w4a16_repack")
+    return out
+
+
+def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qzeros: torch.Tensor | None,
+               group_size: int, zp_bias: int = 8, out: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, stream=None, kernel=None, split_k: int = 0):
+    """out[M, N] = fp16(fp32(a) @ ((q - z) * s)) on the GPU (see include/w4a16.h)."""
+    pa = _dev(a, "a", (torch.float16,))
+    pb = _dev(b_packed, "b_packed", (torch.int32, torch.uint32))
+    ps = _dev(scales, "scales", (torch.float16,))
+    pz = _dev(qzeros, "qzeros", (torch.int32, torch.uint32)) if qzeros is not None else None
+    if a.dim() != 2 or b_packed.dim() != 2 or scales.dim() != 2:
+        raise ValueError("a, b_packed and scales must be 2-D")
+    M, K = a.shape
+    N = b_packed.shape[1] * 8
+    if b_packed.shape[0] != K:
+        raise ValueError("b_packed must be [K, N/8]")
+    if tuple(scales.shape) != (K // group_size, N):
+        raise ValueError("scales must be [K/G, N]")
+    if qzeros is not None and tuple(qzeros.shape) != (K // group_size, N // 8):
+        raise ValueError("qzeros must be [K/G, N/8]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
+    po = _dev(out, "out", (torch.float16,))
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be [M, N]")
+    if workspace is None:
+        workspace = alloc_workspace(M, N, K, group_size, a.device, kernel, split_k)
+    pw = _dev(workspace, "workspace", (torch.uint8,))
+    o = _opts(kernel, split_k)
+    args = (pa, pb, ps, pz, M, N, K, group_size, zp_bias, po, pw, workspace.numel(), _stream_ptr(stream))
+    rc = lib.w4a16_gemm(*args) if o is None else lib.w4a16_gemm_ex(*args, o)
+    _check(rc, "w4a16_gemm")
+    return out
+
+
+def w4a16_workspace_status(workspace: torch.Tensor, clear: bool = False, stream=None) -> int:
+    """Device status word of a GEMM workspace (synchronises the stream)."""
+    v = ctypes.c_int32(-1)
+    _check(lib.w4a16_workspace_status(ctypes.c_void_p(workspace.data_ptr()), int(clear), ctypes.byref(v),
+                                      _stream_ptr(stream)), "w4a16_workspace_status")
+    return int(v.value)

@@ -1,0 +1,230 @@
+// C ABI of the W4A16 library: host-side argument checks, kernel selection and
+// launch. Declarations and the full contract are in include/w4a16.h.
+#include "common.cuh"
+
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+
+namespace w4a16 {
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+void set_error(const char* fmt, const char* detail) {
+    snprintf(g_last_error, sizeof(g_last_error), fmt, detail);
+}
+
+w4a16_status fail_arg(const char* why) {
+    set_error("invalid argument: %s", why);
+    return W4A16_ERR_INVALID_ARG;
+}
+
+w4a16_status fail_cuda(cudaError_t e) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return W4A16_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];   // 0 = not cached yet
+std::atomic<int> g_cc_major[kMaxDevices];
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* p, size_t pn, const void* q, size_t qn) {
+    if (!p || !q || pn == 0 || qn == 0) return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return a < b + qn && b < a + pn;
+}
+
+// Query (once per device) the SM count and compute-capability major.
+cudaError_t device_info(int* sm_count, int* cc_major) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    int sms = g_sm_count[dev].load(std::memory_order_relaxed);
+    int maj = g_cc_major[dev].load(std::memory_order_relaxed);
+    if (sms == 0) {
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e != cudaSuccess) return e;
+        g_cc_major[dev].store(maj, std::memory_order_relaxed);
+        g_sm_count[dev].store(sms, std::memory_order_relaxed);
+    }
+    *sm_count = sms;
+    *cc_major = maj;
+    return cudaSuccess;
+}
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+
+// Shape rules shared by the GEMM entry points; returns nullptr when they hold.
+const char* check_gemm_shape(int64_t M, int64_t N, int64_t K, int32_t G) {
+    if (M < 1) return "M must be >= 1";
+    if (N < 8 || N % 8) return "N must be a positive multiple of 8";
+    if (G < 16 || G % 16) return "group_size must be a positive multiple of 16";
+    if (K < G || K % G) return "K must be a positive multiple of group_size";
+    if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return "dimension too large";
+    return nullptr;
+}
+
+int max_vec_for(const void* b) {
+    return aligned(b, 16) ? 4 : aligned(b, 8) ? 2 : 1;
+}
+
+struct Choice {
+    int kernel;  // W4A16_KERNEL_GEMV or W4A16_KERNEL_TC
+    GemvPlan gemv;
+};
+
+Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms,
+              const void* b) {
+    Choice c{};
+    const int req = opts ? opts->kernel : W4A16_KERNEL_AUTO;
+    // The tensor-core path is selected for M >= 9 once it is available; the
+    // CUDA-core GEMV serves every M until then.
+    c.kernel = (req == W4A16_KERNEL_TC) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
+    c.gemv = plan_gemv(M, N, K, G, opts ? opts->split_k : 0, sms, b ? max_vec_for(b) : 4);
+    return c;
+}
+
+}  // namespace
+
+int device_sm_count(int* err) {
+    int sms = 0, maj = 0;
+    cudaError_t e = device_info(&sms, &maj);
+    if (err) *err = (int)e;
+    return sms;
+}
+
+}  // namespace w4a16
+
+using namespace w4a16;
+
+extern "C" {
+
+const char* w4a16_status_string(w4a16_status s) {
+    switch (s) {
+        case W4A16_OK: return "ok";
+        case W4A16_ERR_INVALID_ARG: return "invalid argument";
+        case W4A16_ERR_UNSUPPORTED: return "unsupported";
+        case W4A16_ERR_CUDA: return "CUDA error";
+        case W4A16_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char* w4a16_last_error(void) { return g_last_error; }
+
+w4a16_status w4a16_repack(const void* ckpt_nk8, void* out_kn8, int64_t N, int64_t K, void* stream) {
+    g_last_error[0] = 0;
+    if (!ckpt_nk8 || !out_kn8) return fail_arg("NULL pointer");
+    if (N < 8 || N % 8) return fail_arg("N must be a positive multiple of 8");
+    if (K < 8 || K % 8) return fail_arg("K must be a positive multiple of 8");
+    if (N >= kMaxDim || K >= kMaxDim) return fail_arg("dimension too large");
+    if (!aligned(ckpt_nk8, 4) || !aligned(out_kn8, 4)) return fail_arg("pointers must be 4-byte aligned");
+    const size_t bytes = (size_t)N * (size_t)K / 2;
+    if (overlaps(ckpt_nk8, bytes, out_kn8, bytes)) return fail_arg("input and output overlap");
+    int sms = 0, maj = 0;
+    cudaError_t e = device_info(&sms, &maj);
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (maj != 10) {
+        set_error("unsupported: %s", "this library is built for sm_100 (B200) devices");
+        return W4A16_ERR_UNSUPPORTED;
+    }
+    e = launch_repack(static_cast<const uint32_t*>(ckpt_nk8), static_cast<uint32_t*>(out_kn8), N, K,
+                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
+}
+
+size_t w4a16_gemm_ex_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size,
+                                     const w4a16_gemm_options* opts) {
+    if (check_gemm_shape(M, N, K, group_size)) return 0;
+    int sms = 0, maj = 0;
+    if (device_info(&sms, &maj) != cudaSuccess) return 0;
+    Choice c = choose(M, N, K, group_size, opts, sms, nullptr);
+    return c.gemv.ws_bytes;
+}
+
+size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size) {
+    return w4a16_gemm_ex_workspace_bytes(M, N, K, group_size, nullptr);
+}
+
+w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scales, const void* qzeros,
+                           int64_t M, int64_t N, int64_t K, int32_t group_size, int32_t zp_bias,
+                           void* out, void* workspace, size_t workspace_bytes, void* stream,
+                           const w4a16_gemm_options* opts) {
+    g_last_error[0] = 0;
+    if (!a || !b_packed || !scales || !out) return fail_arg("NULL pointer");
+    if (const char* why = check_gemm_shape(M, N, K, group_size)) return fail_arg(why);
+    if (!qzeros && (zp_bias < 0 || zp_bias > 15)) return fail_arg("zp_bias must be in 0..15");
+    if (opts && (opts->kernel < W4A16_KERNEL_AUTO || opts->kernel > W4A16_KERNEL_TC))
+        return fail_arg("unknown kernel option");
+    if (opts && (opts->split_k < 0 || opts->split_k > 256)) return fail_arg("split_k must be in 0..256");
+    if (!aligned(a, 2) || !aligned(scales, 2) || !aligned(out, 2)) return fail_arg("fp16 pointers must be 2-byte aligned");
+    if (!aligned(b_packed, 4) || (qzeros && !aligned(qzeros, 4))) return fail_arg("int32 pointers must be 4-byte aligned");
+    const size_t a_bytes = (size_t)M * K * 2, b_bytes = (size_t)K * N / 2, s_bytes = (size_t)(K / group_size) * N * 2;
+    const size_t z_bytes = qzeros ? (size_t)(K / group_size) * N / 2 : 0, o_bytes = (size_t)M * N * 2;
+    if (overlaps(out, o_bytes, a, a_bytes) || overlaps(out, o_bytes, b_packed, b_bytes) ||
+        overlaps(out, o_bytes, scales, s_bytes) || overlaps(out, o_bytes, qzeros, z_bytes))
+        return fail_arg("out overlaps an input");
+
+    int sms = 0, maj = 0;
+    cudaError_t e = device_info(&sms, &maj);
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (maj != 10) {
+        set_error("unsupported: %s", "this library is built for sm_100 (B200) devices");
+        return W4A16_ERR_UNSUPPORTED;
+    }
+    Choice c = choose(M, N, K, group_size, opts, sms, b_packed);
+    if (c.kernel == W4A16_KERNEL_TC) {
+        set_error("unsupported: %s", "tensor-core kernel not available in this build");
+        return W4A16_ERR_UNSUPPORTED;
+    }
+    // The workspace requirement is computed with full vector width; a narrower
+    // plan (misaligned weights) never needs more.
+    const size_t need = c.gemv.ws_bytes;
+    if (need > 0) {
+        if (!workspace) return fail_arg("workspace required (see w4a16_gemm_workspace_bytes)");
+        if (!aligned(workspace, 256)) return fail_arg("workspace must be 256-byte aligned");
+        if (workspace_bytes < need) return fail_arg("workspace too small");
+        if (overlaps(workspace, need, out, o_bytes) || overlaps(workspace, need, a, a_bytes) ||
+            overlaps(workspace, need, b_packed, b_bytes) || overlaps(workspace, need, scales, s_bytes) ||
+            overlaps(workspace, need, qzeros, z_bytes))
+            return fail_arg("workspace overlaps an input or the output");
+    }
+    if (gemv_smem_bytes(M, K, c.gemv.split_k) > 160 * 1024) return fail_arg("split_k too small for this K");
+    e = launch_gemv(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
+                    static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K,
+                    group_size, zp_bias, static_cast<__half*>(out), workspace, c.gemv,
+                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
+}
+
+w4a16_status w4a16_gemm(const void* a, const void* b_packed, const void* scales, const void* qzeros,
+                        int64_t M, int64_t N, int64_t K, int32_t group_size, int32_t zp_bias,
+                        void* out, void* workspace, size_t workspace_bytes, void* stream) {
+    return w4a16_gemm_ex(a, b_packed, scales, qzeros, M, N, K, group_size, zp_bias, out, workspace,
+                         workspace_bytes, stream, nullptr);
+}
+
+w4a16_status w4a16_workspace_status(void* workspace, int32_t clear, int32_t* status, void* stream) {
+    g_last_error[0] = 0;
+    if (!workspace || !status) return fail_arg("NULL pointer");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && clear) {
+        e = cudaMemsetAsync(workspace, 0, sizeof(int32_t), st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
+    if (e != cudaSuccess) return fail_cuda(e);
+    *status = v;
+    return W4A16_OK;
+}
+
+}  // extern "C"
