@@ -38,6 +38,10 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "W4A16 achieved HBM GB/s (M=1) and TFLOP/s (M=32) as fraction of roofline"
+WORKLOADS = {
+    "decode_m1": "decode GEMV M=1 K=4096 N=14336 G=128 sym zp_bias=8 (8B MLP-up shape)",
+    "batch32": "batch-32 GEMM M=32 K=4096 N=14336 G=128 asym, weights repacked from [N,K/8]",
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 
@@ -162,7 +166,8 @@ class Problem:
                           workspace=self.ws, stream=stream)
 
     def launches_per_step(self):
-        return 1 if self.M <= 8 else (self.M + 7) // 8
+        # GEMV for M <= 8; tensor-core GEMM (one launch per 128 rows) above.
+        return 1 if self.M <= 8 else (self.M + 127) // 128
 
 
 def copies_for(bytes_per_copy):
@@ -233,8 +238,14 @@ def run_gpu(args):
     import weight_only_int4_08_b200 as w
     peaks, peak_src = load_peaks()
 
-    case = synth.config2()
-    prob = Problem(w, torch, case, copies_for(alg_bytes(1, case["K"], case["N"], case["G"], False)))
+    if args.workload == "batch32":
+        # batch-32 asymmetric GEMM (tensor cores), weights repacked from the checkpoint layout
+        case = synth.config4()
+        b_kn8 = w.w4a16_repack(to_dev(case["ckpt"], torch), case["N"], case["K"])
+        prob = Problem(w, torch, case, copies_for(alg_bytes(32, case["K"], case["N"], case["G"], True)), b=b_kn8)
+    else:
+        case = synth.config2()
+        prob = Problem(w, torch, case, copies_for(alg_bytes(1, case["K"], case["N"], case["G"], False)))
     K_steps, W_steps = args.steps, args.warmup
 
     # warm-up: W untimed steps
@@ -282,7 +293,7 @@ def run_gpu(args):
     # e2e: through the public API with pinned host buffers; H2D of the step's
     # activations and D2H of its output inside the timed region, every step.
     a_host = torch.from_numpy(np.ascontiguousarray(case["a"])).pin_memory()
-    out_host = torch.empty((1, case["N"]), dtype=torch.float16).pin_memory()
+    out_host = torch.empty((case["M"], case["N"]), dtype=torch.float16).pin_memory()
     a_dev = torch.empty_like(prob.a)
     e2e_steps = min(max(K_steps, 50), 2000)
 
@@ -290,7 +301,7 @@ def run_gpu(args):
         a_dev.copy_(a_host, non_blocking=True)
         j = prob.i % len(prob.bs)
         prob.i += 1
-        w.w4a16_gemm(a_dev, prob.bs[j], prob.ss[j], None, prob.G, prob.zp, out=prob.out, workspace=prob.ws)
+        w.w4a16_gemm(a_dev, prob.bs[j], prob.ss[j], prob.zs[j], prob.G, prob.zp, out=prob.out, workspace=prob.ws)
         out_host.copy_(prob.out, non_blocking=True)
 
     for _ in range(5):
@@ -315,7 +326,8 @@ def run_gpu(args):
     per_launch = measure_problem(torch, prob, 256, 40)
     achieved = prob.bytes / per_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
-    traffic = traffic_from_profiles("gemv_m1_k4096_n14336")
+    kernel_name = "tc_gemm_kernel<32>" if args.workload == "batch32" else "gemv_tma_kernel<1,2>"
+    traffic = traffic_from_profiles("tc_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
 
     extras = {}
     if rank == 0 and not args.no_extras:
@@ -339,7 +351,7 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "fp16 in, fp32 accumulate (int4 weights)",
         "data": "synthetic (seeded; shapes and distributions of the 8B MLP-up decode GEMV)",
-        "config": {"workload": "decode GEMV M=1 K=4096 N=14336 G=128 sym zp_bias=8 (8B MLP-up shape)",
+        "config": {"workload": WORKLOADS[args.workload],
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {len(prob.bs)} rotating weight copies "
                          f"({len(prob.bs) * prob.bytes / 1e6:.0f} MB)",
@@ -347,7 +359,7 @@ def run_gpu(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
-                     "kernel": "gemv_kernel<1,4>", "alg_bytes_per_launch": prob.bytes,
+                     "kernel": kernel_name, "alg_bytes_per_launch": prob.bytes,
                      "us_per_launch": round(per_launch * 1e6, 3)},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": int(a_host.numel() * 2),
                 "d2h_bytes_per_step": int(out_host.numel() * 2), "steps": e2e_steps},
@@ -421,7 +433,7 @@ def run_stack(torch, w, peaks):
         t_roof = max(byts / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
         res[f"config5_stack_M{M}"] = {"us": round(t * 1e6, 1), "GB/s": round(byts / t / 1e9, 1),
                                       "TFLOP/s": round(flops / t / 1e12, 2), "roofline_us": round(t_roof * 1e6, 1),
-                                      "frac_of_roofline": round(t_roof / t, 4), "launches": 128 * (1 if M <= 8 else (M + 7) // 8)}
+                                      "frac_of_roofline": round(t_roof / t, 4), "launches": 128}
         del g
     return res
 
@@ -481,6 +493,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--workload", default="decode_m1", choices=["decode_m1", "batch32"],
+                    help="headline problem: the M=1 decode GEMV (default) or the batch-32 GEMM")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

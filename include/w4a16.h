@@ -123,16 +123,29 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
                         void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Kernel selection for tests and measurement. kernel: W4A16_KERNEL_AUTO uses
- * the same table as w4a16_gemm; GEMV forces the CUDA-core GEMV (any M; M > 8
- * runs it once per 8-row block of A); TC forces the tensor-core GEMM.
- * split_k: 0 = automatic, else the number of K slices (1..256) the GEMV splits
- * its work into (ignored by the tensor-core GEMM).
+ * Kernel selection for tests and measurement.
+ *   kernel: W4A16_KERNEL_AUTO uses the same table as w4a16_gemm (GEMV for
+ *     M <= 8, tensor cores for M >= 9 when N % 128 == 0, K % 64 == 0 and a,
+ *     b_packed are 16-byte aligned); GEMV forces the CUDA-core GEMV (any M;
+ *     M > 8 runs it once per 8-row block of A); TC forces the tensor-core GEMM
+ *     (any M; UNSUPPORTED when the shape or alignment rules above fail).
+ *   split_k: 0 = automatic, else the number of K slices (1..256) the kernel
+ *     splits its work into (the tensor-core GEMM clamps it to K/64).
+ *   debug_flags: 0 in normal use. W4A16_DEBUG_STALL_LOADS makes the kernels'
+ *     load issuers issue nothing, so every device-side wait runs out: the call
+ *     then leaves W4A16_ERR_TIMEOUT in the workspace status word (read it with
+ *     w4a16_workspace_status) and its output undefined. For testing the
+ *     timeout path only.
+ *   wait_limit_us: 0 = the default limit (2 s) on every device-side wait,
+ *     else that many microseconds.
  */
 enum { W4A16_KERNEL_AUTO = 0, W4A16_KERNEL_GEMV = 1, W4A16_KERNEL_TC = 2 };
+enum { W4A16_DEBUG_STALL_LOADS = 1 };
 typedef struct {
     int32_t kernel;
     int32_t split_k;
+    uint32_t debug_flags;
+    uint32_t wait_limit_us;
 } w4a16_gemm_options;
 
 /* Workspace bytes for w4a16_gemm_ex with these options (NULL opts = automatic). */

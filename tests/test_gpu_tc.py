@@ -1,0 +1,102 @@
+"""GPU parity of the tensor-core (tcgen05/TMEM) GEMM and the device-side timeout path.
+
+The tensor-core kernel must satisfy |gpu - oracle| <= 1e-3 + 8e-3 |oracle| on the
+batch workloads (M = 16 of the small-batch sweep, M = 32 with repack) and on
+shapes that exercise every row-block size, group size and split. The timeout
+tests make every device-side wait run out on purpose (the load issuers issue
+nothing) and check that the status word reports it and the context stays usable.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from test_gpu_parity import assert_close, dev, ref, run
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def w():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import weight_only_int4_08_b200 as mod
+    return mod
+
+
+def test_config3_m16_auto_uses_tensor_cores(w):
+    c = synth.config3(16)
+    assert_close(run(w, c), ref(c), "config3 M=16")
+    assert_close(run(w, c, kernel=w.KERNEL_TC), ref(c), "config3 M=16 forced")
+
+
+def test_config4_m32_tensor_cores(w):
+    c = synth.config4()
+    b_dev = w.w4a16_repack(dev(c["ckpt"]), c["N"], c["K"])
+    c["b"] = oracle.repack(c["ckpt"], c["N"], c["K"])
+    assert_close(run(w, c, b=b_dev, kernel=w.KERNEL_TC), ref(c), "config4 TC")
+
+
+@pytest.mark.parametrize("M", [1, 5, 9, 17, 31, 33, 48, 64, 100, 128, 129, 200])
+def test_tc_row_blocks(w, M):
+    c = synth.make_case(M, 512, 384, 128, sym=(M % 2 == 0), seed=100 + M)
+    assert_close(run(w, c, kernel=w.KERNEL_TC), ref(c), f"TC M={M}")
+
+
+@pytest.mark.parametrize("G", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("split", [1, 3])
+def test_tc_group_sizes_and_splits(w, G, split):
+    c = synth.make_case(24, 1024, 256, G, sym=False, seed=G + split)
+    assert_close(run(w, c, kernel=w.KERNEL_TC, split_k=split), ref(c), f"TC G={G} split={split}")
+
+
+@pytest.mark.parametrize("split", [2, 5, 7, 16])
+def test_tc_splits(w, split):
+    c = synth.make_case(32, 2048, 1024, 128, sym=True, seed=split)
+    assert_close(run(w, c, kernel=w.KERNEL_TC, split_k=split), ref(c), f"TC split={split}")
+
+
+def test_tc_q_equals_z_gives_exact_zero(w):
+    K, N, G = 512, 256, 128
+    g = np.random.default_rng(4)
+    zq = synth.words_nibbles_in(g, (K // G, N // 8), 0, 15)
+    c = dict(a=synth.fp16_normal(g, (20, K)), b=np.repeat(zq, G, axis=0),
+             s=synth.fp16_uniform(g, (K // G, N), 0.01, 0.02), z=zq, G=G, zp_bias=0)
+    assert torch.all(run(w, c, kernel=w.KERNEL_TC) == 0)
+
+
+def test_tc_repeatable_and_workspace_restored(w):
+    c = synth.make_case(32, 4096, 2048, 128, sym=False, seed=8)
+    ws = w.alloc_workspace(32, 2048, 4096, 128, kernel=w.KERNEL_TC, split_k=4)
+    o1 = run(w, c, kernel=w.KERNEL_TC, split_k=4, workspace=ws)
+    o2 = run(w, c, kernel=w.KERNEL_TC, split_k=4, workspace=ws)
+    assert torch.equal(o1, o2)
+    assert int(ws[256:256 + 4 * (2048 // 128)].count_nonzero()) == 0
+    assert w.w4a16_workspace_status(ws) == 0
+    assert_close(o1, ref(c), "TC split 4")
+
+
+def test_tc_rejects_unsupported_shapes(w):
+    c = synth.make_case(16, 512, 136, 128, sym=True, seed=9)   # N % 128 != 0
+    with pytest.raises(w.W4A16Error) as e:
+        run(w, c, kernel=w.KERNEL_TC)
+    assert e.value.status == w.W4A16_ERR_UNSUPPORTED
+    # auto falls back to the GEMV row blocks for the same shape
+    assert_close(run(w, c), ref(c), "auto fallback")
+
+
+@pytest.mark.parametrize("kernel,M", [("TC", 32), ("GEMV", 1), ("GEMV", 4)])
+def test_timeout_status_and_recovery(w, kernel, M):
+    """Every device-side wait runs out (nothing is loaded): the kernel must report
+    W4A16_ERR_TIMEOUT in the workspace status word, free its resources and leave
+    the context usable for the next, normal call."""
+    kid = w.KERNEL_TC if kernel == "TC" else w.KERNEL_GEMV
+    c = synth.make_case(M, 1024, 1024, 128, sym=False, seed=11)
+    ws = w.alloc_workspace(M, 1024, 1024, 128, kernel=kid)
+    run(w, c, kernel=kid, workspace=ws, debug_flags=w.DEBUG_STALL_LOADS, wait_limit_us=20000)
+    assert w.w4a16_workspace_status(ws, clear=True) == w.W4A16_ERR_TIMEOUT
+    assert w.w4a16_workspace_status(ws) == 0
+    # counters may be left mid-count by the aborted call: start from a clean workspace
+    ws.zero_()
+    assert_close(run(w, c, kernel=kid, workspace=ws), ref(c), f"after timeout ({kernel})")

@@ -26,7 +26,11 @@ KERNEL_AUTO, KERNEL_GEMV, KERNEL_TC = 0, 1, 2
 
 
 class W4A16Options(ctypes.Structure):
-    _fields_ = [("kernel", ctypes.c_int32), ("split_k", ctypes.c_int32)]
+    _fields_ = [("kernel", ctypes.c_int32), ("split_k", ctypes.c_int32), ("debug_flags", ctypes.c_uint32),
+                ("wait_limit_us", ctypes.c_uint32)]
+
+
+DEBUG_STALL_LOADS = 1
 
 
 _p, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
@@ -80,10 +84,11 @@ def _dev(t, name, dtype):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _opts(kernel, split_k):
-    if kernel is None and not split_k:
+def _opts(kernel, split_k, debug_flags=0, wait_limit_us=0):
+    if kernel is None and not split_k and not debug_flags and not wait_limit_us:
         return None
-    return ctypes.byref(W4A16Options(int(kernel or KERNEL_AUTO), int(split_k or 0)))
+    return ctypes.byref(W4A16Options(int(kernel or KERNEL_AUTO), int(split_k or 0), int(debug_flags),
+                                     int(wait_limit_us)))
 
 
 def w4a16_status_string(status: int) -> str:
@@ -119,7 +124,8 @@ def w4a16_repack(ckpt_nk8: torch.Tensor, N: int, K: int, out: torch.Tensor | Non
 
 def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qzeros: torch.Tensor | None,
                group_size: int, zp_bias: int = 8, out: torch.Tensor | None = None,
-               workspace: torch.Tensor | None = None, stream=None, kernel=None, split_k: int = 0):
+               workspace: torch.Tensor | None = None, stream=None, kernel=None, split_k: int = 0,
+               debug_flags: int = 0, wait_limit_us: int = 0):
     """out[M, N] = fp16(fp32(a) @ ((q - z) * s)) on the GPU (see include/w4a16.h)."""
     pa = _dev(a, "a", (torch.float16,))
     pb = _dev(b_packed, "b_packed", (torch.int32, torch.uint32))
@@ -143,7 +149,7 @@ def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qz
     if workspace is None:
         workspace = alloc_workspace(M, N, K, group_size, a.device, kernel, split_k)
     pw = _dev(workspace, "workspace", (torch.uint8,))
-    o = _opts(kernel, split_k)
+    o = _opts(kernel, split_k, debug_flags, wait_limit_us)
     args = (pa, pb, ps, pz, M, N, K, group_size, zp_bias, po, pw, workspace.numel(), _stream_ptr(stream))
     rc = lib.w4a16_gemm(*args) if o is None else lib.w4a16_gemm_ex(*args, o)
     _check(rc, "w4a16_gemm")

@@ -50,7 +50,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         for _, err in results:
             sys.stderr.write(err)
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *[o for o, _ in results], "-o", tmp, "-lcuda"]
+    cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *[o for o, _ in results], "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")

@@ -1,6 +1,7 @@
 // Internal declarations shared by the library's translation units (not installed).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -16,7 +17,15 @@ namespace w4a16 {
 constexpr size_t kWsHeader = 256;
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Device-side wait policy for the pipelined kernels: the limit on each wait,
+// and (tests only) a switch that makes the load issuers issue nothing.
+struct WaitPolicy {
+    uint64_t limit_ns;
+    int stall_loads;
+};
+
 struct GemvPlan {
+    bool tma;         // TMA-fed kernel (N % 32 == 0, 16-byte aligned weights) or plain loads
     int vec;          // int32 words per thread per row (4, 2 or 1)
     int m_rows;       // activation rows handled by one launch (1..8)
     int split_k;      // CTAs along K per column tile
@@ -25,19 +34,43 @@ struct GemvPlan {
     size_t counters_off, partials_off;
 };
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the library
+// does not link libcuda, so it loads on machines without a driver).
+cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank, void* gaddr,
+                              const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                              const cuuint32_t* estrides, CUtensorMapSwizzle swizzle);
+
 // SM count of the current device (cached per device).
 int device_sm_count(int* err);
 
-// max_vec: widest packed-word vector (4, 2, 1) the weight pointer's alignment allows.
-GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count, int max_vec);
+// max_vec: widest packed-word vector (4, 2, 1) the weight pointer's alignment allows;
+// tma_ok: the caller allows the TMA-fed kernel.
+GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count, int max_vec,
+                   bool tma_ok);
 
 // Largest rows-per-CTA slab the GEMV stages in shared memory for an explicit split.
 size_t gemv_smem_bytes(int64_t M, int64_t K, int split_k);
+
+struct TcPlan {
+    int mblk_max;     // activation rows per launch (<= 128)
+    int mn;           // MMA N: rows padded to a multiple of 16
+    int n_tiles;      // N / 128
+    int split_k;      // CTAs along K per tile
+    size_t ws_bytes;  // workspace bytes (status word + counters + partials)
+    size_t counters_off, partials_off;
+};
+
+// The tensor-core kernel needs N % 128 == 0, K % 64 == 0 and 16-byte aligned A and weights.
+bool tc_supported(int64_t M, int64_t N, int64_t K, int32_t G, const void* a, const void* b);
+TcPlan plan_tc(int64_t M, int64_t N, int64_t K, int32_t G, int sm_count, int split_k_request);
+cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M, int64_t N,
+                      int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace, const TcPlan& plan,
+                      const WaitPolicy& wp, cudaStream_t st);
 
 cudaError_t launch_repack(const uint32_t* ckpt, uint32_t* out, int64_t N, int64_t K, cudaStream_t st);
 
 cudaError_t launch_gemv(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z,
                         int64_t M, int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out,
-                        void* workspace, const GemvPlan& plan, cudaStream_t st);
+                        void* workspace, const GemvPlan& plan, const WaitPolicy& wp, cudaStream_t st);
 
 }  // namespace w4a16

@@ -1,0 +1,507 @@
+// Tensor-core (tcgen05 / TMEM) W4A16 GEMM for M >= 9 activation rows.
+//
+// Operation (vLLM PR #37352 analysis page, "코드 분석 1", `_w4a16_reference`):
+//   out[m, n] = fp16( sum_g s[g, n] * sum_{k in g} a[m, k] * (q[k, n] - z[g, n]) ),
+// fp32 accumulation. The weights are the big operand, so the MMA is "swapped":
+// the MMA's M dimension is N (128 output columns per CTA, one per TMEM lane),
+// its N dimension is the activation rows (padded to MN, a multiple of 16), and
+//   D[n, m] += A[n, k] * B[k, m],  A = (q - z)^T from TMEM, B = activations^T.
+//
+// (q - z) is an integer in [-15, 15]: exact in fp16, and its products with the
+// fp16 activations are exact in the fp32 accumulator, so each group's partial
+// sum D_g is exact up to fp32 summation; the fp16 scale is applied in fp32 when
+// D_g is read back (tot += s[g, n] * D_g), never rounded into the weights.
+//
+// Roles (one CTA = one 128-column tile x one K slab; 10 warps):
+//   warp 4      producer: per stage of 64 k-rows, 64 one-row bulk copies of the
+//               tile's packed words (64 B each) into a staggered shared-memory
+//               layout, and one 2-D TMA load of the activation tile [MN x 64]
+//               (128-byte swizzle, the canonical K-major layout of operand B);
+//   warps 0-3   dequantisers: warp p owns TMEM lanes 32p..32p+31; each thread
+//               turns 4 k-rows x 4 columns of nibbles into exact fp16 (q - z)
+//               pairs (byte permute + 0x6400 magic + fp16 subtract) and writes
+//               them to TMEM with tcgen05.st.16x256b;
+//   warp 5      TMEM allocator and MMA issuer: tcgen05.mma.kind::f16 with A
+//               from TMEM and B from shared memory, 4 per stage (K = 16 each);
+//               a fresh accumulator per group segment, double-buffered, and a
+//               tcgen05.commit to an mbarrier at each segment end;
+//   warps 6-9   epilogue: tcgen05.ld of each finished group segment, scaled by
+//               s[g, n] in fp32 into register totals; then the fp16 output, or
+//               the fp32 split-K partial and the last-CTA ordered reduction.
+// Every mbarrier wait is bounded; a wait that runs out sets the workspace
+// status word to W4A16_ERR_TIMEOUT, and all roles drain and leave, freeing TMEM.
+//
+// Lane/column bookkeeping: dequantiser thread t of warp p (t0 = t % 4,
+// t1 = t / 4) writes TMEM lanes {t1, t1+8, t1+16, t1+24} (+32p), which hold tile
+// columns {4 t1, 4 t1 + 1, 4 t1 + 2, 4 t1 + 3} (+32p): lane L holds column
+// 32p + 4 (L % 8) + L / 8. Columns at odd nibble positions come out of the
+// unpack scaled by 16 (exact), undone in the epilogue.
+#include "common.cuh"
+#include "ptx.cuh"
+
+#include <algorithm>
+#include <atomic>
+
+namespace w4a16 {
+namespace {
+
+constexpr int kBlockN = 128;                    // MMA M = TMEM lanes = output columns per CTA
+constexpr int kTileWords = kBlockN / 8;         // 16 packed words per k-row of the tile
+constexpr int kStageK = 64;                     // k-rows per pipeline stage
+constexpr int kWPitch = 128;                    // shared bytes per staged weight row (64 used)
+constexpr int kWStageBytes = kStageK * kWPitch;
+constexpr int kTmemStages = 4;                  // A slots in TMEM (32 columns = 64 k each)
+constexpr int kThreadsTC = 320;
+
+template <int MN>
+struct TcCfg {
+    static constexpr int kSmemStages = MN <= 32 ? 8 : (MN <= 64 ? 6 : 4);
+    static constexpr int kBStageBytes = MN * 128;           // MN rows x 64 k x 2 B
+    static constexpr int kDCol = kTmemStages * 32;          // first accumulator column
+    static constexpr int kColsNeeded = kDCol + 2 * MN;
+    static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64 : kColsNeeded <= 128 ? 128
+                                   : kColsNeeded <= 256 ? 256 : 512;
+    static constexpr size_t kSmemBytes = 1024 /*align slack*/ + (size_t)kSmemStages * (kBStageBytes + kWStageBytes);
+};
+
+struct TcArgs {
+    const uint32_t* b;     // [K, N/8]
+    const __half* s;       // [K/G, N]
+    const uint32_t* z;     // [K/G, N/8] or nullptr
+    __half* out;           // [M, N] (already offset to this row block)
+    float* partials;       // [split][mblk][N]
+    uint32_t* counters;    // [n_tiles]
+    int* status;           // workspace status word
+    int64_t N, K;
+    int G, zp_bias, split, mblk, m0;
+    int stall_loads;       // tests only: the producer issues nothing (every wait runs out)
+    uint64_t wait_ns;      // limit on each device-side wait
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile in the 128-byte
+// swizzle layout: rows of 64 fp16 (128 B), 8-row atoms 1024 B apart.
+__device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4)      // start address, 16-byte units
+         | ((uint64_t)1 << 16)                       // leading byte offset (unused for this layout)
+         | ((uint64_t)(1024 >> 4) << 32)             // stride byte offset: 8 rows x 128 B
+         | ((uint64_t)1 << 46)                       // descriptor version (sm_100)
+         | ((uint64_t)2 << 61);                      // 128-byte swizzle
+}
+
+// Instruction descriptor: fp16 A and B (K-major), fp32 D, M = 128, N = MN.
+template <int MN>
+__device__ __forceinline__ uint32_t idesc_f16() {
+    return (1u << 4) | ((uint32_t)(MN >> 3) << 17) | ((uint32_t)(kBlockN >> 4) << 24);
+}
+
+// Segments of 16-k MMA steps: a segment ends at a group end or at the slab end.
+struct SegIter {
+    int64_t k_lo, k_hi;  // slab rows
+    int G;
+    __device__ bool starts(int64_t k) const { return k == k_lo || k % G == 0; }
+    __device__ bool ends(int64_t k) const { return k + 16 == k_hi || (k + 16) % G == 0; }
+};
+
+template <int MN>
+__global__ void __launch_bounds__(kThreadsTC, (TcCfg<MN>::kTmemCols <= 256 && MN <= 32) ? 2 : 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, TcArgs p) {
+    using C = TcCfg<MN>;
+    constexpr int SS = C::kSmemStages;
+    extern __shared__ __align__(1024) unsigned char s_raw[];
+    unsigned char* s_base = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(s_raw) + 1023) & ~(uintptr_t)1023);
+    unsigned char* s_b = s_base;                                   // [SS][MN x 128 B], 1024-aligned stages
+    unsigned char* s_w = s_base + (size_t)SS * C::kBStageBytes;    // [SS][64 rows x 128 B]
+
+    __shared__ __align__(8) uint64_t bar_full[SS], bar_empty[SS];
+    __shared__ __align__(8) uint64_t bar_afull[kTmemStages], bar_aempty[kTmemStages];
+    __shared__ __align__(8) uint64_t bar_dfull[2], bar_dempty[2], bar_drain;
+    __shared__ uint32_t s_tmem;
+    __shared__ volatile int s_abort;
+    __shared__ int s_last;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = blockIdx.x;
+    const int64_t nstage_all = p.K / kStageK;
+    const int64_t st_lo = nstage_all * blockIdx.y / p.split, st_hi = nstage_all * (blockIdx.y + 1) / p.split;
+    const int nst = (int)(st_hi - st_lo);
+    const SegIter seg{st_lo * kStageK, st_hi * kStageK, p.G};
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int i = 0; i < SS; ++i) {
+            ptx::mbar_init(ptx::smem_addr(&bar_full[i]), 1);
+            ptx::mbar_init(ptx::smem_addr(&bar_empty[i]), 1);
+        }
+        for (int i = 0; i < kTmemStages; ++i) {
+            ptx::mbar_init(ptx::smem_addr(&bar_afull[i]), 128);
+            ptx::mbar_init(ptx::smem_addr(&bar_aempty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(ptx::smem_addr(&bar_dfull[i]), 1);
+            ptx::mbar_init(ptx::smem_addr(&bar_dempty[i]), 128);
+        }
+        ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
+        ptx::mbar_fence_init();
+    }
+    if (warp == 5) {
+        ptx::tmem_alloc(ptx::smem_addr(&s_tmem), C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            ptx::prefetch_tensormap(&amap);
+            const int64_t nw = p.N / 8;
+            const uint32_t tx = kStageK * kTileWords * 4 + C::kBStageBytes;
+            int issued = 0;
+            for (int i = 0; i < nst && !p.stall_loads; ++i) {
+                const int s = i % SS;
+                if (!ptx::mbar_wait(ptx::smem_addr(&bar_empty[s]), ((i / SS) & 1) ^ 1, &s_abort, p.wait_ns)) break;
+                const uint32_t full = ptx::smem_addr(&bar_full[s]);
+                ptx::mbar_arrive_expect_tx(full, tx);
+                const int64_t k0 = (st_lo + i) * kStageK;
+                const uint32_t* src = p.b + k0 * nw + (int64_t)tile * kTileWords;
+                const uint32_t wdst = ptx::smem_addr(s_w + (size_t)s * kWStageBytes);
+                for (int r = 0; r < kStageK; ++r)
+                    ptx::bulk_g2s(wdst + r * kWPitch + 16 * ((r >> 2) & 3), src + r * nw, kTileWords * 4, full);
+                ptx::tma_load_2d(ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes), &amap, (int32_t)k0, p.m0, full);
+                issued = i + 1;
+            }
+            if (s_abort) {  // let copies already issued land before the CTA leaves
+                volatile int dummy = 0;
+                for (int i = max(0, issued - SS); i < issued; ++i)
+                    ptx::mbar_wait(ptx::smem_addr(&bar_full[i % SS]), (i / SS) & 1, &dummy, p.wait_ns);
+            }
+        }
+    } else if (warp < 4) {
+        // -------------------------------------------------------- dequantisers
+        const int t0 = lane & 3, t1 = lane >> 2;
+        const int cw = 4 * warp + (t1 >> 1);                 // packed word (of 16) holding my 4 columns
+        const int b0 = 2 * (t1 & 1), b1 = b0 + 1;            // its bytes: columns (0,1) and (2,3) of mine
+        const uint32_t sel0 = (uint32_t)(b0 | (b0 << 4) | ((4 + b0) << 8) | ((4 + b0) << 12));
+        const uint32_t sel1 = (uint32_t)(b1 | (b1 << 4) | ((4 + b1) << 8) | ((4 + b1) << 12));
+        const int64_t nw = p.N / 8;
+        const int64_t word = (int64_t)tile * kTileWords + cw;
+        int64_t g_cur = -1;
+        uint32_t bias_lo0 = 0, bias_hi0 = 0, bias_lo1 = 0, bias_hi1 = 0;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+        for (int i = 0; i < nst; ++i) {
+            const int s = i % SS, ts = i % kTmemStages;
+            // Wait outcomes are made warp-uniform: the tcgen05 stores below are .sync.aligned.
+            bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns);
+            okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_aempty[ts]), ((i / kTmemStages) & 1) ^ 1, &s_abort,
+                                        p.wait_ns);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            ptx::tc_fence_after();
+            const unsigned char* wst = s_w + (size_t)s * kWStageBytes + 16 * t0 + 4 * cw;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t kk = (st_lo + i) * kStageK + 16 * j;
+                const int64_t g = kk / p.G;
+                if (g != g_cur) {
+                    g_cur = g;
+                    uint32_t z0, z1, z2, z3;
+                    if (p.z) {
+                        const uint32_t zw = __ldg(p.z + g * nw + word);
+                        z0 = (zw >> (8 * b0)) & 0xFu;
+                        z1 = (zw >> (8 * b0 + 4)) & 0xFu;
+                        z2 = (zw >> (8 * b1)) & 0xFu;
+                        z3 = (zw >> (8 * b1 + 4)) & 0xFu;
+                    } else {
+                        z0 = z1 = z2 = z3 = (uint32_t)p.zp_bias;
+                    }
+                    // (1024 + z) for low-nibble columns, (1024 + 16 z) for high ones, in both halves
+                    bias_lo0 = (0x6400u + z0) * 0x00010001u;
+                    bias_hi0 = (0x6400u + 16u * z1) * 0x00010001u;
+                    bias_lo1 = (0x6400u + z2) * 0x00010001u;
+                    bias_hi1 = (0x6400u + 16u * z3) * 0x00010001u;
+                }
+                // rows 16j + 4 t0 + {0..3}; row r sits at r * 128 + 16 * ((r >> 2) & 3) = ... + 16 t0
+                const unsigned char* rp = wst + (16 * j + 4 * t0) * kWPitch;
+                const uint32_t w0 = *reinterpret_cast<const uint32_t*>(rp);
+                const uint32_t w1 = *reinterpret_cast<const uint32_t*>(rp + kWPitch);
+                const uint32_t w2 = *reinterpret_cast<const uint32_t*>(rp + 2 * kWPitch);
+                const uint32_t w3 = *reinterpret_cast<const uint32_t*>(rp + 3 * kWPitch);
+                const uint32_t x01 = prmt(w0, w1, sel0), x23 = prmt(w2, w3, sel0);
+                const uint32_t y01 = prmt(w0, w1, sel1), y23 = prmt(w2, w3, sel1);
+                const uint32_t col = (uint32_t)(ts * 32 + 8 * j);
+                ptx::tmem_st_16x256b(lane_base + col,
+                                     hsub2((x01 & 0x000F000Fu) | 0x64006400u, bias_lo0),
+                                     hsub2((x23 & 0x000F000Fu) | 0x64006400u, bias_lo0),
+                                     hsub2((x01 & 0x00F000F0u) | 0x64006400u, bias_hi0),
+                                     hsub2((x23 & 0x00F000F0u) | 0x64006400u, bias_hi0));
+                ptx::tmem_st_16x256b(lane_base + (16u << 16) + col,
+                                     hsub2((y01 & 0x000F000Fu) | 0x64006400u, bias_lo1),
+                                     hsub2((y23 & 0x000F000Fu) | 0x64006400u, bias_lo1),
+                                     hsub2((y01 & 0x00F000F0u) | 0x64006400u, bias_hi1),
+                                     hsub2((y23 & 0x00F000F0u) | 0x64006400u, bias_hi1));
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_addr(&bar_afull[ts]));
+        }
+    } else if (warp == 5) {
+        // ----------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f16<MN>();
+            int sg = 0;              // segment counter
+            uint32_t acc = 0;
+            for (int i = 0; i < nst; ++i) {
+                const int s = i % SS, ts = i % kTmemStages;
+                if (!ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort, p.wait_ns)) break;
+                if (!ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns)) break;
+                ptx::tc_fence_after();
+                const uint32_t bbase = ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes);
+                bool ok = true;
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t k = (st_lo + i) * kStageK + 16 * j;
+                    const int db = sg & 1;
+                    if (seg.starts(k)) {
+                        if (!ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1, &s_abort, p.wait_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        acc = 0;
+                    }
+                    ptx::mma_f16_ts(tmem + (uint32_t)(C::kDCol + db * MN), tmem + (uint32_t)(ts * 32 + 8 * j),
+                                    kmajor_sw128_desc(bbase + 32 * j), idesc, acc);
+                    acc = 1;
+                    if (seg.ends(k)) {
+                        ptx::mma_commit(ptx::smem_addr(&bar_dfull[db]));
+                        ++sg;
+                    }
+                }
+                ptx::mma_commit(ptx::smem_addr(&bar_empty[s]));
+                ptx::mma_commit(ptx::smem_addr(&bar_aempty[ts]));
+                if (!ok) break;
+            }
+            // Wait for every MMA issued above before TMEM can be released.
+            volatile int dummy = 0;
+            ptx::mma_commit(ptx::smem_addr(&bar_drain));
+            ptx::mbar_wait(ptx::smem_addr(&bar_drain), 0, &dummy, p.wait_ns);
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue
+        const int sub = warp & 3;                           // TMEM lanes 32 sub .. 32 sub + 31
+        const int et = threadIdx.x - 192;                   // 0..127 within the epilogue warps
+        const int ncol = 32 * sub + 4 * (lane & 7) + (lane >> 3);
+        const int64_t n = (int64_t)tile * kBlockN + ncol;
+        const float fscale = (lane >> 3) & 1 ? 0.0625f : 1.0f;
+        float tot[MN];
+#pragma unroll
+        for (int m = 0; m < MN; ++m) tot[m] = 0.f;
+        int sg = 0;
+        bool ok = true;
+        for (int64_t k = seg.k_lo; k < seg.k_hi && ok; k += 16) {
+            if (!seg.ends(k)) continue;
+            // segment [k_start, k + 16) just ended; its group is (k / G)
+            const int db = sg & 1;
+            const float sc = fscale * __half2float(p.s[(k / p.G) * p.N + n]);
+            const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_dfull[db]), (sg >> 1) & 1, &s_abort, p.wait_ns);
+            if (!__all_sync(0xffffffffu, okw)) {  // warp-uniform: tcgen05.ld is .sync.aligned
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t taddr = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(C::kDCol + db * MN);
+#pragma unroll
+            for (int c0 = 0; c0 < MN; c0 += 16) {
+                uint32_t v[16];
+                ptx::tmem_ld_32x32b_x16(taddr + c0, v);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) tot[c0 + q] = fmaf(sc, __uint_as_float(v[q]), tot[c0 + q]);
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(ptx::smem_addr(&bar_dempty[db]));
+            ++sg;
+        }
+        // One decision for all 128 epilogue threads (a timeout seen by any of them,
+        // or by another role, skips the output), so the named barriers below match.
+        const bool bad = ptx::named_bar_or(1, 128, !ok || s_abort);
+        if (!bad) {
+            if (p.split == 1) {
+#pragma unroll
+                for (int m = 0; m < MN; ++m)
+                    if (m < p.mblk) p.out[(int64_t)m * p.N + n] = __float2half_rn(tot[m]);
+            } else {
+#pragma unroll
+                for (int m = 0; m < MN; ++m)
+                    if (m < p.mblk) p.partials[((int64_t)blockIdx.y * p.mblk + m) * p.N + n] = tot[m];
+                __threadfence();
+                ptx::named_bar_sync(1, 128);
+                if (et == 0) {
+                    const uint32_t ticket = atomicAdd(p.counters + tile, 1u);
+                    s_last = (ticket == (uint32_t)p.split - 1);
+                }
+                ptx::named_bar_sync(1, 128);
+                if (s_last) {
+                    __threadfence();
+                    for (int m = 0; m < p.mblk; ++m) {
+                        float a = 0.f;
+                        for (int y = 0; y < p.split; ++y) a += __ldcg(p.partials + ((int64_t)y * p.mblk + m) * p.N + n);
+                        p.out[(int64_t)m * p.N + n] = __float2half_rn(a);
+                    }
+                    if (et == 0) p.counters[tile] = 0u;
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (s_abort && threadIdx.x == 0 && p.status) atomicExch(p.status, (int)W4A16_ERR_TIMEOUT);
+    if (warp == 5) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+using TcFn = void (*)(CUtensorMap, TcArgs);
+
+TcFn select_tc(int mn) {
+    switch (mn) {
+        case 16: return tc_gemm_kernel<16>;
+        case 32: return tc_gemm_kernel<32>;
+        case 48: return tc_gemm_kernel<48>;
+        case 64: return tc_gemm_kernel<64>;
+        case 80: return tc_gemm_kernel<80>;
+        case 96: return tc_gemm_kernel<96>;
+        case 112: return tc_gemm_kernel<112>;
+        default: return tc_gemm_kernel<128>;
+    }
+}
+
+size_t tc_smem(int mn) {
+    switch (mn) {
+        case 16: return TcCfg<16>::kSmemBytes;
+        case 32: return TcCfg<32>::kSmemBytes;
+        case 48: return TcCfg<48>::kSmemBytes;
+        case 64: return TcCfg<64>::kSmemBytes;
+        case 80: return TcCfg<80>::kSmemBytes;
+        case 96: return TcCfg<96>::kSmemBytes;
+        case 112: return TcCfg<112>::kSmemBytes;
+        default: return TcCfg<128>::kSmemBytes;
+    }
+}
+
+std::atomic<int> g_tc_occ[9];
+
+int tc_ctas_per_sm(int mn) {
+    int n = g_tc_occ[mn / 16].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    TcFn k = select_tc(mn);
+    const size_t smem = tc_smem(mn);
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreadsTC, smem) != cudaSuccess || n < 1) n = 1;
+    // TMEM: at most 512 columns per SM.
+    const int cols = mn <= 64 ? 256 : 512;
+    n = std::min(n, 512 / cols);
+    g_tc_occ[mn / 16].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+}  // namespace
+
+bool tc_supported(int64_t M, int64_t N, int64_t K, int32_t G, const void* a, const void* b) {
+    (void)M; (void)G;
+    return N % kBlockN == 0 && K % kStageK == 0 && (reinterpret_cast<uintptr_t>(a) % 16) == 0 &&
+           (reinterpret_cast<uintptr_t>(b) % 16) == 0;
+}
+
+TcPlan plan_tc(int64_t M, int64_t N, int64_t K, int32_t G, int sm_count, int split_k_request) {
+    (void)G;
+    TcPlan pl{};
+    pl.mblk_max = (int)std::min<int64_t>(M, 128);
+    pl.mn = (int)((pl.mblk_max + 15) / 16 * 16);
+    pl.n_tiles = (int)(N / kBlockN);
+    const int64_t nst = K / kStageK;
+    const int64_t slots = (int64_t)std::max(sm_count, 1) * tc_ctas_per_sm(pl.mn);
+    // Pick the split that fills whole waves best, counting the fp32 partials
+    // it writes and reads as extra traffic against the packed weights.
+    double best = -1.0;
+    int best_s = 1;
+    for (int s = 1; s <= 16 && s <= nst; ++s) {
+        const int64_t ctas = (int64_t)pl.n_tiles * s;
+        const double waves = (double)((ctas + slots - 1) / slots);
+        const double fill = (double)ctas / (waves * slots);
+        const double wbytes = (double)K * N / 2;
+        const double pbytes = s > 1 ? 2.0 * s * pl.mblk_max * (double)N * 4 : 0.0;
+        const double score = fill * wbytes / (wbytes + pbytes);
+        if (score > best + 1e-9) {
+            best = score;
+            best_s = s;
+        }
+    }
+    pl.split_k = split_k_request > 0 ? (int)std::min<int64_t>(split_k_request, nst) : best_s;
+    pl.counters_off = kWsHeader;
+    pl.partials_off = align_up(kWsHeader + (size_t)pl.n_tiles * 4, 256);
+    pl.ws_bytes = pl.partials_off + (pl.split_k > 1 ? (size_t)pl.split_k * pl.mblk_max * (size_t)N * 4 : 0);
+    return pl;
+}
+
+cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M, int64_t N,
+                      int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace, const TcPlan& pl,
+                      const WaitPolicy& wp, cudaStream_t st) {
+    // Tensor map over the activations [M, K] fp16: box 64 k x MN rows, 128-byte swizzle;
+    // rows past M read as zero.
+    CUtensorMap amap;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kStageK, (cuuint32_t)pl.mn};
+    const cuuint32_t estr[2] = {1, 1};
+    cudaError_t e = encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)a, dims, strides, box, estr,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    char* ws = static_cast<char*>(workspace);
+    for (int64_t m0 = 0; m0 < M; m0 += 128) {
+        TcArgs args;
+        args.b = b;
+        args.s = s;
+        args.z = z;
+        args.out = out + m0 * N;
+        args.partials = reinterpret_cast<float*>(ws + pl.partials_off);
+        args.counters = reinterpret_cast<uint32_t*>(ws + pl.counters_off);
+        args.status = reinterpret_cast<int*>(ws);
+        args.N = N;
+        args.K = K;
+        args.G = G;
+        args.zp_bias = zp_bias;
+        args.split = pl.split_k;
+        args.mblk = (int)std::min<int64_t>(128, M - m0);
+        args.m0 = (int)m0;
+        args.stall_loads = wp.stall_loads;
+        args.wait_ns = wp.limit_ns;
+        // Every row block uses the plan's MN (the largest); a short last block
+        // leaves its padded rows to TMA's zero fill.
+        TcFn k = select_tc(pl.mn);
+        const size_t smem = tc_smem(pl.mn);
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k<<<dim3((unsigned)pl.n_tiles, (unsigned)pl.split_k), kThreadsTC, smem, st>>>(amap, args);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace w4a16

@@ -78,20 +78,68 @@ int max_vec_for(const void* b) {
 struct Choice {
     int kernel;  // W4A16_KERNEL_GEMV or W4A16_KERNEL_TC
     GemvPlan gemv;
+    TcPlan tc;
 };
 
+// Kernel table: the CUDA-core GEMV for M <= 8, the tensor-core GEMM for M >= 9
+// when the shape and pointers allow it (N % 128, K % 64, 16-byte aligned A and
+// weights), the GEMV's 8-row blocks otherwise. Null pointers (workspace query)
+// count as aligned.
 Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms,
-              const void* b) {
+              const void* a, const void* b) {
     Choice c{};
     const int req = opts ? opts->kernel : W4A16_KERNEL_AUTO;
-    // The tensor-core path is selected for M >= 9 once it is available; the
-    // CUDA-core GEMV serves every M until then.
-    c.kernel = (req == W4A16_KERNEL_TC) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
-    c.gemv = plan_gemv(M, N, K, G, opts ? opts->split_k : 0, sms, b ? max_vec_for(b) : 4);
+    const bool tc_ok = tc_supported(M, N, K, G, a ? a : (const void*)16, b ? b : (const void*)16);
+    if (req == W4A16_KERNEL_TC) c.kernel = W4A16_KERNEL_TC;
+    else if (req == W4A16_KERNEL_GEMV) c.kernel = W4A16_KERNEL_GEMV;
+    else c.kernel = (M >= 9 && tc_ok) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
+    if (c.kernel == W4A16_KERNEL_TC) {
+        if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, opts ? opts->split_k : 0);
+    } else {
+        c.gemv = plan_gemv(M, N, K, G, opts ? opts->split_k : 0, sms, b ? max_vec_for(b) : 4, true);
+    }
     return c;
 }
 
+// Workspace that covers every plan this shape can take, whatever the alignment
+// of the pointers turns out to be at launch.
+size_t ws_bound(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms) {
+    size_t ws = 0;
+    const int req = opts ? opts->kernel : W4A16_KERNEL_AUTO;
+    if (req != W4A16_KERNEL_TC) {
+        const int split = opts ? opts->split_k : 0;
+        for (int v : {4, 2, 1})
+            for (bool tma : {true, false}) ws = std::max(ws, plan_gemv(M, N, K, G, split, sms, v, tma).ws_bytes);
+    }
+    const bool tc_shape = tc_supported(M, N, K, G, (const void*)16, (const void*)16);
+    if (tc_shape && (req == W4A16_KERNEL_TC || (req == W4A16_KERNEL_AUTO && M >= 9)))
+        ws = std::max(ws, plan_tc(M, N, K, G, sms, opts ? opts->split_k : 0).ws_bytes);
+    return ws;
+}
+
 }  // namespace
+
+cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank, void* gaddr,
+                              const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                              const cuuint32_t* estrides, CUtensorMapSwizzle swizzle) {
+    using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static std::atomic<EncodeFn> fn{nullptr};
+    EncodeFn f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+        f = reinterpret_cast<EncodeFn>(p);
+        fn.store(f, std::memory_order_release);
+    }
+    CUresult r = f(map, dtype, rank, gaddr, dims, strides, box, estrides, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 
 int device_sm_count(int* err) {
     int sms = 0, maj = 0;
@@ -145,8 +193,7 @@ size_t w4a16_gemm_ex_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t gr
     if (check_gemm_shape(M, N, K, group_size)) return 0;
     int sms = 0, maj = 0;
     if (device_info(&sms, &maj) != cudaSuccess) return 0;
-    Choice c = choose(M, N, K, group_size, opts, sms, nullptr);
-    return c.gemv.ws_bytes;
+    return ws_bound(M, N, K, group_size, opts, sms);
 }
 
 size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size) {
@@ -164,6 +211,7 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
     if (opts && (opts->kernel < W4A16_KERNEL_AUTO || opts->kernel > W4A16_KERNEL_TC))
         return fail_arg("unknown kernel option");
     if (opts && (opts->split_k < 0 || opts->split_k > 256)) return fail_arg("split_k must be in 0..256");
+    if (opts && (opts->debug_flags & ~(uint32_t)W4A16_DEBUG_STALL_LOADS)) return fail_arg("unknown debug flag");
     if (!aligned(a, 2) || !aligned(scales, 2) || !aligned(out, 2)) return fail_arg("fp16 pointers must be 2-byte aligned");
     if (!aligned(b_packed, 4) || (qzeros && !aligned(qzeros, 4))) return fail_arg("int32 pointers must be 4-byte aligned");
     const size_t a_bytes = (size_t)M * K * 2, b_bytes = (size_t)K * N / 2, s_bytes = (size_t)(K / group_size) * N * 2;
@@ -179,14 +227,12 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
         set_error("unsupported: %s", "this library is built for sm_100 (B200) devices");
         return W4A16_ERR_UNSUPPORTED;
     }
-    Choice c = choose(M, N, K, group_size, opts, sms, b_packed);
-    if (c.kernel == W4A16_KERNEL_TC) {
-        set_error("unsupported: %s", "tensor-core kernel not available in this build");
+    Choice c = choose(M, N, K, group_size, opts, sms, a, b_packed);
+    if (c.kernel == W4A16_KERNEL_TC && !tc_supported(M, N, K, group_size, a, b_packed)) {
+        set_error("unsupported: %s", "tensor-core kernel needs N % 128 == 0, K % 64 == 0, 16-byte aligned a and b_packed");
         return W4A16_ERR_UNSUPPORTED;
     }
-    // The workspace requirement is computed with full vector width; a narrower
-    // plan (misaligned weights) never needs more.
-    const size_t need = c.gemv.ws_bytes;
+    const size_t need = c.kernel == W4A16_KERNEL_TC ? c.tc.ws_bytes : c.gemv.ws_bytes;
     if (need > 0) {
         if (!workspace) return fail_arg("workspace required (see w4a16_gemm_workspace_bytes)");
         if (!aligned(workspace, 256)) return fail_arg("workspace must be 256-byte aligned");
@@ -196,11 +242,20 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
             overlaps(workspace, need, qzeros, z_bytes))
             return fail_arg("workspace overlaps an input or the output");
     }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    WaitPolicy wp;
+    wp.limit_ns = (opts && opts->wait_limit_us) ? (uint64_t)opts->wait_limit_us * 1000ull : 2000000000ull;
+    wp.stall_loads = (opts && (opts->debug_flags & W4A16_DEBUG_STALL_LOADS)) ? 1 : 0;
+    if (c.kernel == W4A16_KERNEL_TC) {
+        e = launch_tc(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
+                      static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K, group_size,
+                      zp_bias, static_cast<__half*>(out), workspace, c.tc, wp, st);
+        return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
+    }
     if (gemv_smem_bytes(M, K, c.gemv.split_k) > 160 * 1024) return fail_arg("split_k too small for this K");
     e = launch_gemv(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
                     static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K,
-                    group_size, zp_bias, static_cast<__half*>(out), workspace, c.gemv,
-                    static_cast<cudaStream_t>(stream));
+                    group_size, zp_bias, static_cast<__half*>(out), workspace, c.gemv, wp, st);
     return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
 }
 
