@@ -167,6 +167,40 @@ W4A16_API w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const 
  */
 W4A16_API w4a16_status w4a16_workspace_status(void* workspace, int32_t clear, int32_t* status, void* stream);
 
+/*
+ * w4a16_gemm_noalloc — w4a16_gemm for callers that cannot allocate device memory.
+ *
+ * The page has no counterpart: this entry point is an addition of this library.
+ * Some callers cannot hand over a workspace: code that must not call cudaMalloc
+ * because it can synchronise the whole device in the middle of a latency-
+ * critical loop, or code embedded in a program whose device memory belongs to
+ * another allocator. This variant runs the CUDA-core GEMV kernel family (any M;
+ * M > 8 in 8-row blocks) with its scratch memory — status word, split-K
+ * counters and fp32 partials — in a fixed array compiled into the library
+ * (w4a16_noalloc_scratch_bytes() bytes, 8 MiB) instead of a workspace. It
+ * allocates nothing and calls no allocating routine.
+ *
+ *   Arguments a .. out and stream: as for w4a16_gemm (no workspace arguments).
+ *   Limit: a shape whose GEMV scratch need exceeds the fixed array returns
+ *     W4A16_ERR_INVALID_ARG ("needs N bytes of scratch...") and launches nothing.
+ *   Every GPU that loads the library holds the array until the process exits.
+ *   The first call on a device looks up the array's device address with that
+ *     device current (cudaGetSymbolAddress) and caches it; make that first call
+ *     before any stream capture.
+ *   Each call first clears the array's status word and counters on `stream`
+ *     (cudaMemsetAsync), then launches the kernel on `stream`.
+ *   All calls share the one array: calls that overlap on the GPU (different
+ *     streams without ordering, or several host threads) race and give wrong
+ *     results. Order them on one stream or with events.
+ * Errors: as w4a16_gemm; CUDA when the address lookup or the clear fails.
+ */
+W4A16_API w4a16_status w4a16_gemm_noalloc(const void* a, const void* b_packed, const void* scales,
+                                          const void* qzeros, int64_t M, int64_t N, int64_t K, int32_t group_size,
+                                          int32_t zp_bias, void* out, void* stream);
+
+/* Size in bytes of the fixed scratch array used by w4a16_gemm_noalloc. */
+W4A16_API size_t w4a16_noalloc_scratch_bytes(void);
+
 /* Static description of a status code. Never NULL. */
 W4A16_API const char* w4a16_status_string(w4a16_status s);
 

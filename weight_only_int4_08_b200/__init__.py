@@ -47,13 +47,18 @@ lib.w4a16_gemm_ex.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _i32, _p, 
 lib.w4a16_gemm_ex.restype = ctypes.c_int
 lib.w4a16_workspace_status.argtypes = [_p, _i32, ctypes.POINTER(ctypes.c_int32), _p]
 lib.w4a16_workspace_status.restype = ctypes.c_int
+lib.w4a16_gemm_noalloc.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _i32, _p, _p]
+lib.w4a16_gemm_noalloc.restype = ctypes.c_int
+lib.w4a16_noalloc_scratch_bytes.argtypes = []
+lib.w4a16_noalloc_scratch_bytes.restype = _sz
 lib.w4a16_status_string.argtypes = [ctypes.c_int]
 lib.w4a16_status_string.restype = ctypes.c_char_p
 lib.w4a16_last_error.argtypes = []
 lib.w4a16_last_error.restype = ctypes.c_char_p
 
 EXPORTED = ("w4a16_repack", "w4a16_gemm_workspace_bytes", "w4a16_gemm", "w4a16_gemm_ex_workspace_bytes",
-            "w4a16_gemm_ex", "w4a16_workspace_status", "w4a16_status_string", "w4a16_last_error")
+            "w4a16_gemm_ex", "w4a16_workspace_status", "w4a16_status_string", "w4a16_last_error",
+            "w4a16_gemm_noalloc", "w4a16_noalloc_scratch_bytes")
 
 
 class W4A16Error(RuntimeError):
@@ -153,6 +158,24 @@ def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qz
     args = (pa, pb, ps, pz, M, N, K, group_size, zp_bias, po, pw, workspace.numel(), _stream_ptr(stream))
     rc = lib.w4a16_gemm(*args) if o is None else lib.w4a16_gemm_ex(*args, o)
     _check(rc, "w4a16_gemm")
+    return out
+
+
+def w4a16_gemm_noalloc(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qzeros: torch.Tensor | None,
+                       group_size: int, zp_bias: int = 8, out: torch.Tensor | None = None, stream=None):
+    """w4a16_gemm without a workspace: scratch comes from the library's fixed array
+    (for callers that cannot allocate device memory; see include/w4a16.h)."""
+    pa = _dev(a, "a", (torch.float16,))
+    pb = _dev(b_packed, "b_packed", (torch.int32, torch.uint32))
+    ps = _dev(scales, "scales", (torch.float16,))
+    pz = _dev(qzeros, "qzeros", (torch.int32, torch.uint32)) if qzeros is not None else None
+    M, K = a.shape
+    N = b_packed.shape[1] * 8
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
+    po = _dev(out, "out", (torch.float16,))
+    _check(lib.w4a16_gemm_noalloc(pa, pb, ps, pz, M, N, K, group_size, zp_bias, po, _stream_ptr(stream)),
+           "w4a16_gemm_noalloc")
     return out
 
 

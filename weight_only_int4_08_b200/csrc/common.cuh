@@ -40,6 +40,9 @@ cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuin
                               const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
                               const cuuint32_t* estrides, CUtensorMapSwizzle swizzle);
 
+// Record the text returned by w4a16_last_error() on the calling thread.
+void set_last_error(const char* msg);
+
 // SM count of the current device (cached per device).
 int device_sm_count(int* err);
 

@@ -141,6 +141,8 @@ cudaError_t encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, cuuin
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 int device_sm_count(int* err) {
     int sms = 0, maj = 0;
     cudaError_t e = device_info(&sms, &maj);
