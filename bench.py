@@ -326,7 +326,7 @@ def run_gpu(args):
     per_launch = measure_problem(torch, prob, 256, 40)
     achieved = prob.bytes / per_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
-    kernel_name = "tc_gemm_kernel<32>" if args.workload == "batch32" else "gemv_tma_kernel<1,2>"
+    kernel_name = "tc_gemm_kernel<32>" if args.workload == "batch32" else "gemv_mma_kernel<1>"
     traffic = traffic_from_profiles("tc_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
 
     extras = {}

@@ -126,9 +126,12 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  * Kernel selection for tests and measurement.
  *   kernel: W4A16_KERNEL_AUTO uses the same table as w4a16_gemm (GEMV for
  *     M <= 8, tensor cores for M >= 9 when N % 128 == 0, K % 64 == 0 and a,
- *     b_packed are 16-byte aligned); GEMV forces the CUDA-core GEMV (any M;
- *     M > 8 runs it once per 8-row block of A); TC forces the tensor-core GEMM
- *     (any M; UNSUPPORTED when the shape or alignment rules above fail).
+ *     b_packed are 16-byte aligned); GEMV forces the GEMV family (any M; M > 8
+ *     runs it once per 8-row block of A): its multiply-accumulate uses warp
+ *     mma.sync when N % 32 == 0, b_packed is 16-byte and a 4-byte aligned, the
+ *     CUDA-core fp32 loop otherwise; GEMV_FMA forces the CUDA-core fp32 loop;
+ *     TC forces the tensor-core GEMM (any M; UNSUPPORTED when the shape or
+ *     alignment rules above fail).
  *   split_k: 0 = automatic, else the number of K slices (1..256) the kernel
  *     splits its work into (the tensor-core GEMM clamps it to K/64).
  *   debug_flags: 0 in normal use. W4A16_DEBUG_STALL_LOADS makes the kernels'
@@ -139,7 +142,7 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  *   wait_limit_us: 0 = the default limit (2 s) on every device-side wait,
  *     else that many microseconds.
  */
-enum { W4A16_KERNEL_AUTO = 0, W4A16_KERNEL_GEMV = 1, W4A16_KERNEL_TC = 2 };
+enum { W4A16_KERNEL_AUTO = 0, W4A16_KERNEL_GEMV = 1, W4A16_KERNEL_TC = 2, W4A16_KERNEL_GEMV_FMA = 3 };
 enum { W4A16_DEBUG_STALL_LOADS = 1 };
 typedef struct {
     int32_t kernel;

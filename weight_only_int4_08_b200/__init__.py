@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 lib = ctypes.CDLL(LIB_PATH)
 
 W4A16_OK, W4A16_ERR_INVALID_ARG, W4A16_ERR_UNSUPPORTED, W4A16_ERR_CUDA, W4A16_ERR_TIMEOUT = range(5)
-KERNEL_AUTO, KERNEL_GEMV, KERNEL_TC = 0, 1, 2
+KERNEL_AUTO, KERNEL_GEMV, KERNEL_TC, KERNEL_GEMV_FMA = 0, 1, 2, 3
 
 
 class W4A16Options(ctypes.Structure):

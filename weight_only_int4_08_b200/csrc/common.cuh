@@ -25,6 +25,7 @@ struct WaitPolicy {
 };
 
 struct GemvPlan {
+    bool mma;         // tensor-instruction (mma.sync) inner loop, or the CUDA-core fp32 one
     bool tma;         // TMA-fed kernel (N % 32 == 0, 16-byte aligned weights) or plain loads
     int vec;          // int32 words per thread per row (4, 2 or 1)
     int m_rows;       // activation rows handled by one launch (1..8)
@@ -50,6 +51,13 @@ int device_sm_count(int* err);
 // tma_ok: the caller allows the TMA-fed kernel.
 GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count, int max_vec,
                    bool tma_ok);
+
+// The mma.sync GEMV: N % 32 == 0, 16-byte aligned weights, 4-byte aligned activations.
+bool gemv_mma_supported(int64_t N, const void* a, const void* b);
+GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count);
+cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M,
+                            int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace,
+                            const GemvPlan& plan, const WaitPolicy& wp, cudaStream_t st);
 
 // Largest rows-per-CTA slab the GEMV stages in shared memory for an explicit split.
 size_t gemv_smem_bytes(int64_t M, int64_t K, int split_k);

@@ -49,6 +49,9 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxRowsPerCta = 1024;          // bounds the staged activations
 constexpr int kRing = 4;                      // TMA stages per warp
 constexpr int kStageBytes = 2048;             // bytes per TMA stage
+#ifndef W4A16_GEMV_SCALAR_FMA
+#define W4A16_GEMV_SCALAR_FMA 0               // 1: scalar fp32 add/FMA instead of the packed forms
+#endif
 #ifndef W4A16_GEMV_M1_VEC
 #define W4A16_GEMV_M1_VEC 2                   // packed words per lane for one activation row
 #endif
@@ -147,7 +150,14 @@ __device__ __forceinline__ void accumulate_row(float2 (&gacc)[MT][4 * V], const 
     for (int v = 0; v < V; ++v) {
         unpack_raw(wv[v], d[v]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) d[v][i] = __fadd2_rn(d[v][i], gm.nz[v][i]);
+        for (int i = 0; i < 4; ++i) {
+#if W4A16_GEMV_SCALAR_FMA
+            d[v][i].x += gm.nz[v][i].x;
+            d[v][i].y += gm.nz[v][i].y;
+#else
+            d[v][i] = __fadd2_rn(d[v][i], gm.nz[v][i]);
+#endif
+        }
     }
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
@@ -155,7 +165,14 @@ __device__ __forceinline__ void accumulate_row(float2 (&gacc)[MT][4 * V], const 
 #pragma unroll
         for (int v = 0; v < V; ++v)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) gacc[m][4 * v + i] = __ffma2_rn(av, d[v][i], gacc[m][4 * v + i]);
+            for (int i = 0; i < 4; ++i) {
+#if W4A16_GEMV_SCALAR_FMA
+                gacc[m][4 * v + i].x = fmaf(av.x, d[v][i].x, gacc[m][4 * v + i].x);
+                gacc[m][4 * v + i].y = fmaf(av.x, d[v][i].y, gacc[m][4 * v + i].y);
+#else
+                gacc[m][4 * v + i] = __ffma2_rn(av, d[v][i], gacc[m][4 * v + i]);
+#endif
+            }
     }
 }
 

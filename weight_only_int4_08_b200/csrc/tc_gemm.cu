@@ -13,14 +13,15 @@
 // D_g is read back (tot += s[g, n] * D_g), never rounded into the weights.
 //
 // Roles (one CTA = one 128-column tile x one K slab; 10 warps):
-//   warp 4      producer: per stage of 64 k-rows, 64 one-row bulk copies of the
-//               tile's packed words (64 B each) into a staggered shared-memory
-//               layout, and one 2-D TMA load of the activation tile [MN x 64]
-//               (128-byte swizzle, the canonical K-major layout of operand B);
-//   warps 0-3   dequantisers: warp p owns TMEM lanes 32p..32p+31; each thread
-//               turns 4 k-rows x 4 columns of nibbles into exact fp16 (q - z)
-//               pairs (byte permute + 0x6400 magic + fp16 subtract) and writes
-//               them to TMEM with tcgen05.st.16x256b;
+//   warp 4      producer: per stage of 64 k-rows, one 2-D TMA load of the
+//               tile's packed words [64 rows x 64 B] (64-byte swizzle) and one of
+//               the activation tile [MN x 64] (128-byte swizzle, the canonical
+//               K-major layout of operand B);
+//   warps 0-3   dequantisers: warp p owns TMEM lanes 32p..32p+31 and tile
+//               columns 32p..32p+31 (one 16-byte chunk of each weight row);
+//               ldmatrix.trans hands every thread two k-rows of 4 columns per
+//               register, which become exact fp16 (q - z) pairs (0x6400 magic +
+//               fp16 subtract) written to TMEM with tcgen05.st.16x128b;
 //   warp 5      TMEM allocator and MMA issuer: tcgen05.mma.kind::f16 with A
 //               from TMEM and B from shared memory, 4 per stage (K = 16 each);
 //               a fresh accumulator per group segment, double-buffered, and a
@@ -32,10 +33,12 @@
 // status word to W4A16_ERR_TIMEOUT, and all roles drain and leave, freeing TMEM.
 //
 // Lane/column bookkeeping: dequantiser thread t of warp p (t0 = t % 4,
-// t1 = t / 4) writes TMEM lanes {t1, t1+8, t1+16, t1+24} (+32p), which hold tile
-// columns {4 t1, 4 t1 + 1, 4 t1 + 2, 4 t1 + 3} (+32p): lane L holds column
-// 32p + 4 (L % 8) + L / 8. Columns at odd nibble positions come out of the
-// unpack scaled by 16 (exact), undone in the epilogue.
+// t1 = t / 4) holds tile columns 32p + 4 t1 + {0, 1, 2, 3} (nibbles 4(t1%2)..
+// of packed word 4p + t1/2) and writes them to TMEM lanes {t1, t1+8, t1+16,
+// t1+24} (+32p): lane L holds column 32p + 4 (L % 8) + L / 8. Columns at odd
+// nibble positions come out of the unpack scaled by 16 (exact), undone in the
+// epilogue. The thread's k-pair in each 8-row matrix is t0, i.e. TMEM column
+// (k - k_stage) / 2 of the stage's A slot, in natural k order.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -48,8 +51,7 @@ namespace {
 constexpr int kBlockN = 128;                    // MMA M = TMEM lanes = output columns per CTA
 constexpr int kTileWords = kBlockN / 8;         // 16 packed words per k-row of the tile
 constexpr int kStageK = 64;                     // k-rows per pipeline stage
-constexpr int kWPitch = 128;                    // shared bytes per staged weight row (64 used)
-constexpr int kWStageBytes = kStageK * kWPitch;
+constexpr int kWStageBytes = kStageK * kTileWords * 4;   // 64 rows x 64 B, 64-byte swizzle
 constexpr int kTmemStages = 4;                  // A slots in TMEM (32 columns = 64 k each)
 constexpr int kThreadsTC = 320;
 
@@ -77,12 +79,6 @@ struct TcArgs {
     int stall_loads;       // tests only: the producer issues nothing (every wait runs out)
     uint64_t wait_ns;      // limit on each device-side wait
 };
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-    return r;
-}
 
 __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
     uint32_t r;
@@ -116,14 +112,14 @@ struct SegIter {
 
 template <int MN>
 __global__ void __launch_bounds__(kThreadsTC, (TcCfg<MN>::kTmemCols <= 256 && MN <= 32) ? 2 : 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, TcArgs p) {
+tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap, TcArgs p) {
     using C = TcCfg<MN>;
     constexpr int SS = C::kSmemStages;
     extern __shared__ __align__(1024) unsigned char s_raw[];
     unsigned char* s_base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(s_raw) + 1023) & ~(uintptr_t)1023);
     unsigned char* s_b = s_base;                                   // [SS][MN x 128 B], 1024-aligned stages
-    unsigned char* s_w = s_base + (size_t)SS * C::kBStageBytes;    // [SS][64 rows x 128 B]
+    unsigned char* s_w = s_base + (size_t)SS * C::kBStageBytes;    // [SS][64 rows x 64 B], 1024-aligned stages
 
     __shared__ __align__(8) uint64_t bar_full[SS], bar_empty[SS];
     __shared__ __align__(8) uint64_t bar_afull[kTmemStages], bar_aempty[kTmemStages];
@@ -169,20 +165,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, TcArgs p) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             ptx::prefetch_tensormap(&amap);
-            const int64_t nw = p.N / 8;
-            const uint32_t tx = kStageK * kTileWords * 4 + C::kBStageBytes;
+            ptx::prefetch_tensormap(&wmap);
+            const uint32_t tx = kWStageBytes + C::kBStageBytes;
             int issued = 0;
             for (int i = 0; i < nst && !p.stall_loads; ++i) {
                 const int s = i % SS;
                 if (!ptx::mbar_wait(ptx::smem_addr(&bar_empty[s]), ((i / SS) & 1) ^ 1, &s_abort, p.wait_ns)) break;
                 const uint32_t full = ptx::smem_addr(&bar_full[s]);
                 ptx::mbar_arrive_expect_tx(full, tx);
-                const int64_t k0 = (st_lo + i) * kStageK;
-                const uint32_t* src = p.b + k0 * nw + (int64_t)tile * kTileWords;
-                const uint32_t wdst = ptx::smem_addr(s_w + (size_t)s * kWStageBytes);
-                for (int r = 0; r < kStageK; ++r)
-                    ptx::bulk_g2s(wdst + r * kWPitch + 16 * ((r >> 2) & 3), src + r * nw, kTileWords * 4, full);
-                ptx::tma_load_2d(ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes), &amap, (int32_t)k0, p.m0, full);
+                const int32_t k0 = (int32_t)((st_lo + i) * kStageK);
+                ptx::tma_load_2d(ptx::smem_addr(s_w + (size_t)s * kWStageBytes), &wmap, tile * kTileWords, k0, full);
+                ptx::tma_load_2d(ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes), &amap, k0, p.m0, full);
                 issued = i + 1;
             }
             if (s_abort) {  // let copies already issued land before the CTA leaves
@@ -193,15 +186,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, TcArgs p) {
         }
     } else if (warp < 4) {
         // -------------------------------------------------------- dequantisers
-        const int t0 = lane & 3, t1 = lane >> 2;
-        const int cw = 4 * warp + (t1 >> 1);                 // packed word (of 16) holding my 4 columns
-        const int b0 = 2 * (t1 & 1), b1 = b0 + 1;            // its bytes: columns (0,1) and (2,3) of mine
-        const uint32_t sel0 = (uint32_t)(b0 | (b0 << 4) | ((4 + b0) << 8) | ((4 + b0) << 12));
-        const uint32_t sel1 = (uint32_t)(b1 | (b1 << 4) | ((4 + b1) << 8) | ((4 + b1) << 12));
+        const int t1 = lane >> 2;
         const int64_t nw = p.N / 8;
-        const int64_t word = (int64_t)tile * kTileWords + cw;
+        const int64_t word = (int64_t)tile * kTileWords + 4 * warp + (t1 >> 1);  // holds my 4 columns
+        const int nib0 = 4 * (t1 & 1);                                           // their first nibble
         int64_t g_cur = -1;
-        uint32_t bias_lo0 = 0, bias_hi0 = 0, bias_lo1 = 0, bias_hi1 = 0;
+        const int64_t ngroups = p.K / p.G;
+        uint32_t zw_next = 0u;
+        uint32_t bias0 = 0, bias1 = 0, bias2 = 0, bias3 = 0;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
         for (int i = 0; i < nst; ++i) {
             const int s = i % SS, ts = i % kTmemStages;
@@ -211,48 +203,40 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, TcArgs p) {
                                         p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) break;
             ptx::tc_fence_after();
-            const unsigned char* wst = s_w + (size_t)s * kWStageBytes + 16 * t0 + 4 * cw;
+            const uint32_t wbase = ptx::smem_addr(s_w + (size_t)s * kWStageBytes);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int64_t kk = (st_lo + i) * kStageK + 16 * j;
-                const int64_t g = kk / p.G;
-                if (g != g_cur) {
-                    g_cur = g;
-                    uint32_t z0, z1, z2, z3;
-                    if (p.z) {
-                        const uint32_t zw = __ldg(p.z + g * nw + word);
-                        z0 = (zw >> (8 * b0)) & 0xFu;
-                        z1 = (zw >> (8 * b0 + 4)) & 0xFu;
-                        z2 = (zw >> (8 * b1)) & 0xFu;
-                        z3 = (zw >> (8 * b1 + 4)) & 0xFu;
-                    } else {
-                        z0 = z1 = z2 = z3 = (uint32_t)p.zp_bias;
+            for (int h = 0; h < 2; ++h) {
+                // rows 32h .. 32h + 31 as four 8x8 matrices of 16-bit halves; my address row
+                // is 32h + lane; 16-byte chunk `warp` of it, moved by the 64-byte swizzle
+                const int row = 32 * h + lane;
+                uint32_t R[4];
+                ptx::ldmatrix_x4_trans(wbase + row * 64 + 16 * (warp ^ ((row >> 1) & 3)), R);
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) {
+                    const int64_t kk = (st_lo + i) * kStageK + 32 * h + 8 * mi;   // first k of this matrix
+                    const int64_t g = kk / p.G;
+                    if (g != g_cur) {
+                        // zero word of this group (prefetched one group ahead), then prefetch the next
+                        uint32_t zraw = 0u;
+                        if (p.z) {
+                            zraw = (g == g_cur + 1 && g_cur >= 0) ? zw_next : __ldg(p.z + g * nw + word);
+                            if (g + 1 < ngroups) zw_next = __ldg(p.z + (g + 1) * nw + word);
+                        }
+                        g_cur = g;
+                        const uint32_t zw = p.z ? (zraw >> (4 * nib0)) : (uint32_t)p.zp_bias * 0x1111u;
+                        // (1024 + z) for low-nibble columns, (1024 + 16 z) for high ones, in both halves
+                        bias0 = (0x6400u + (zw & 0xFu)) * 0x00010001u;
+                        bias1 = (0x6400u + 16u * ((zw >> 4) & 0xFu)) * 0x00010001u;
+                        bias2 = (0x6400u + ((zw >> 8) & 0xFu)) * 0x00010001u;
+                        bias3 = (0x6400u + 16u * ((zw >> 12) & 0xFu)) * 0x00010001u;
                     }
-                    // (1024 + z) for low-nibble columns, (1024 + 16 z) for high ones, in both halves
-                    bias_lo0 = (0x6400u + z0) * 0x00010001u;
-                    bias_hi0 = (0x6400u + 16u * z1) * 0x00010001u;
-                    bias_lo1 = (0x6400u + z2) * 0x00010001u;
-                    bias_hi1 = (0x6400u + 16u * z3) * 0x00010001u;
+                    const uint32_t x = R[mi], y = x >> 8;
+                    const uint32_t col = (uint32_t)(ts * 32 + 16 * h + 4 * mi);
+                    ptx::tmem_st_16x128b(lane_base + col, hsub2((x & 0x000F000Fu) | 0x64006400u, bias0),
+                                         hsub2((x & 0x00F000F0u) | 0x64006400u, bias1));
+                    ptx::tmem_st_16x128b(lane_base + (16u << 16) + col, hsub2((y & 0x000F000Fu) | 0x64006400u, bias2),
+                                         hsub2((y & 0x00F000F0u) | 0x64006400u, bias3));
                 }
-                // rows 16j + 4 t0 + {0..3}; row r sits at r * 128 + 16 * ((r >> 2) & 3) = ... + 16 t0
-                const unsigned char* rp = wst + (16 * j + 4 * t0) * kWPitch;
-                const uint32_t w0 = *reinterpret_cast<const uint32_t*>(rp);
-                const uint32_t w1 = *reinterpret_cast<const uint32_t*>(rp + kWPitch);
-                const uint32_t w2 = *reinterpret_cast<const uint32_t*>(rp + 2 * kWPitch);
-                const uint32_t w3 = *reinterpret_cast<const uint32_t*>(rp + 3 * kWPitch);
-                const uint32_t x01 = prmt(w0, w1, sel0), x23 = prmt(w2, w3, sel0);
-                const uint32_t y01 = prmt(w0, w1, sel1), y23 = prmt(w2, w3, sel1);
-                const uint32_t col = (uint32_t)(ts * 32 + 8 * j);
-                ptx::tmem_st_16x256b(lane_base + col,
-                                     hsub2((x01 & 0x000F000Fu) | 0x64006400u, bias_lo0),
-                                     hsub2((x23 & 0x000F000Fu) | 0x64006400u, bias_lo0),
-                                     hsub2((x01 & 0x00F000F0u) | 0x64006400u, bias_hi0),
-                                     hsub2((x23 & 0x00F000F0u) | 0x64006400u, bias_hi0));
-                ptx::tmem_st_16x256b(lane_base + (16u << 16) + col,
-                                     hsub2((y01 & 0x000F000Fu) | 0x64006400u, bias_lo1),
-                                     hsub2((y23 & 0x000F000Fu) | 0x64006400u, bias_lo1),
-                                     hsub2((y01 & 0x00F000F0u) | 0x64006400u, bias_hi1),
-                                     hsub2((y23 & 0x00F000F0u) | 0x64006400u, bias_hi1));
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -311,11 +295,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, TcArgs p) {
         for (int m = 0; m < MN; ++m) tot[m] = 0.f;
         int sg = 0;
         bool ok = true;
-        for (int64_t k = seg.k_lo; k < seg.k_hi && ok; k += 16) {
-            if (!seg.ends(k)) continue;
-            // segment [k_start, k + 16) just ended; its group is (k / G)
+        // Segment ends in order; each segment's scale is loaded one segment ahead.
+        auto seg_end_from = [&](int64_t k) -> int64_t {  // last 16-step of the segment holding k
+            return min(seg.k_hi, (k / p.G + 1) * (int64_t)p.G) - 16;
+        };
+        auto scale_of = [&](int64_t kend) -> float {
+            return fscale * __half2float(p.s[(kend / p.G) * p.N + n]);
+        };
+        int64_t k_end = seg_end_from(seg.k_lo);
+        float sc = scale_of(k_end);
+        while (k_end >= seg.k_lo && ok) {
+            const int64_t k_next = k_end + 16 < seg.k_hi ? seg_end_from(k_end + 16) : -1;
+            const float sc_next = k_next >= 0 ? scale_of(k_next) : 0.f;
             const int db = sg & 1;
-            const float sc = fscale * __half2float(p.s[(k / p.G) * p.N + n]);
             const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_dfull[db]), (sg >> 1) & 1, &s_abort, p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) {  // warp-uniform: tcgen05.ld is .sync.aligned
                 ok = false;
@@ -334,6 +326,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, TcArgs p) {
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_addr(&bar_dempty[db]));
             ++sg;
+            k_end = k_next;
+            sc = sc_next;
         }
         // One decision for all 128 epilogue threads (a timeout seen by any of them,
         // or by another role, skips the output), so the named barriers below match.
@@ -376,7 +370,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, TcArgs p) {
     }
 }
 
-using TcFn = void (*)(CUtensorMap, TcArgs);
+using TcFn = void (*)(CUtensorMap, CUtensorMap, TcArgs);
 
 TcFn select_tc(int mn) {
     switch (mn) {
@@ -409,13 +403,19 @@ std::atomic<int> g_tc_occ[9];
 int tc_ctas_per_sm(int mn) {
     int n = g_tc_occ[mn / 16].load(std::memory_order_relaxed);
     if (n > 0) return n;
+    // Resident CTAs per SM from the three budgets the kernel draws on: shared
+    // memory (228 KB per SM, 1 KB reserved per CTA), registers (64 K per SM)
+    // and tensor memory (512 columns per SM).
     TcFn k = select_tc(mn);
     const size_t smem = tc_smem(mn);
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreadsTC, smem) != cudaSuccess || n < 1) n = 1;
-    // TMEM: at most 512 columns per SM.
+    cudaFuncAttributes fa{};
+    int regs = 255;
+    if (cudaFuncGetAttributes(&fa, k) == cudaSuccess && fa.numRegs > 0) regs = fa.numRegs;
+    const int by_smem = (int)((228 * 1024) / (smem + fa.sharedSizeBytes + 1024));
+    const int regs_per_warp = (regs + 7) / 8 * 8 * 32;  // allocation granularity: 8 registers per thread
+    const int by_regs = 65536 / (regs_per_warp * (kThreadsTC / 32));
     const int cols = mn <= 64 ? 256 : 512;
-    n = std::min(n, 512 / cols);
+    n = std::max(1, std::min(std::min(by_smem, by_regs), 512 / cols));
     g_tc_occ[mn / 16].store(n, std::memory_order_relaxed);
     return n;
 }
@@ -472,6 +472,14 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
     cudaError_t e = encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)a, dims, strides, box, estr,
                                       CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
+    // Tensor map over the packed weights [K, N/8] int32: box 16 words x 64 rows, 64-byte swizzle.
+    CUtensorMap wmap;
+    const cuuint64_t wdims[2] = {(cuuint64_t)(N / 8), (cuuint64_t)K};
+    const cuuint64_t wstrides[1] = {(cuuint64_t)(N / 8) * 4};
+    const cuuint32_t wbox[2] = {(cuuint32_t)kTileWords, (cuuint32_t)kStageK};
+    e = encode_tensor_map(&wmap, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, (void*)b, wdims, wstrides, wbox, estr,
+                          CU_TENSOR_MAP_SWIZZLE_64B);
+    if (e != cudaSuccess) return e;
     char* ws = static_cast<char*>(workspace);
     for (int64_t m0 = 0; m0 < M; m0 += 128) {
         TcArgs args;
@@ -497,7 +505,7 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
         const size_t smem = tc_smem(pl.mn);
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        k<<<dim3((unsigned)pl.n_tiles, (unsigned)pl.split_k), kThreadsTC, smem, st>>>(amap, args);
+        k<<<dim3((unsigned)pl.n_tiles, (unsigned)pl.split_k), kThreadsTC, smem, st>>>(amap, wmap, args);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

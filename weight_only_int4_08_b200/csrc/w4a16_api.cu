@@ -91,12 +91,15 @@ Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_optio
     const int req = opts ? opts->kernel : W4A16_KERNEL_AUTO;
     const bool tc_ok = tc_supported(M, N, K, G, a ? a : (const void*)16, b ? b : (const void*)16);
     if (req == W4A16_KERNEL_TC) c.kernel = W4A16_KERNEL_TC;
-    else if (req == W4A16_KERNEL_GEMV) c.kernel = W4A16_KERNEL_GEMV;
+    else if (req == W4A16_KERNEL_GEMV || req == W4A16_KERNEL_GEMV_FMA) c.kernel = W4A16_KERNEL_GEMV;
     else c.kernel = (M >= 9 && tc_ok) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
+    const int split = opts ? opts->split_k : 0;
     if (c.kernel == W4A16_KERNEL_TC) {
-        if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, opts ? opts->split_k : 0);
+        if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, split);
+    } else if (req != W4A16_KERNEL_GEMV_FMA && gemv_mma_supported(N, a ? a : (const void*)16, b ? b : (const void*)16)) {
+        c.gemv = plan_gemv_mma(M, N, K, G, split, sms);
     } else {
-        c.gemv = plan_gemv(M, N, K, G, opts ? opts->split_k : 0, sms, b ? max_vec_for(b) : 4, true);
+        c.gemv = plan_gemv(M, N, K, G, split, sms, b ? max_vec_for(b) : 4, true);
     }
     return c;
 }
@@ -110,6 +113,7 @@ size_t ws_bound(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_opt
         const int split = opts ? opts->split_k : 0;
         for (int v : {4, 2, 1})
             for (bool tma : {true, false}) ws = std::max(ws, plan_gemv(M, N, K, G, split, sms, v, tma).ws_bytes);
+        if (req != W4A16_KERNEL_GEMV_FMA && N % 32 == 0) ws = std::max(ws, plan_gemv_mma(M, N, K, G, split, sms).ws_bytes);
     }
     const bool tc_shape = tc_supported(M, N, K, G, (const void*)16, (const void*)16);
     if (tc_shape && (req == W4A16_KERNEL_TC || (req == W4A16_KERNEL_AUTO && M >= 9)))
@@ -210,7 +214,7 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
     if (!a || !b_packed || !scales || !out) return fail_arg("NULL pointer");
     if (const char* why = check_gemm_shape(M, N, K, group_size)) return fail_arg(why);
     if (!qzeros && (zp_bias < 0 || zp_bias > 15)) return fail_arg("zp_bias must be in 0..15");
-    if (opts && (opts->kernel < W4A16_KERNEL_AUTO || opts->kernel > W4A16_KERNEL_TC))
+    if (opts && (opts->kernel < W4A16_KERNEL_AUTO || opts->kernel > W4A16_KERNEL_GEMV_FMA))
         return fail_arg("unknown kernel option");
     if (opts && (opts->split_k < 0 || opts->split_k > 256)) return fail_arg("split_k must be in 0..256");
     if (opts && (opts->debug_flags & ~(uint32_t)W4A16_DEBUG_STALL_LOADS)) return fail_arg("unknown debug flag");
@@ -238,7 +242,10 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
     if (need > 0) {
         if (!workspace) return fail_arg("workspace required (see w4a16_gemm_workspace_bytes)");
         if (!aligned(workspace, 256)) return fail_arg("workspace must be 256-byte aligned");
-        if (workspace_bytes < need) return fail_arg("workspace too small");
+        // The documented contract: at least what the size query advertises for these arguments
+        // (a bound over the kernels the automatic choice may take), not just what this plan uses.
+        if (workspace_bytes < std::max(need, ws_bound(M, N, K, group_size, opts, sms)))
+            return fail_arg("workspace too small");
         if (overlaps(workspace, need, out, o_bytes) || overlaps(workspace, need, a, a_bytes) ||
             overlaps(workspace, need, b_packed, b_bytes) || overlaps(workspace, need, scales, s_bytes) ||
             overlaps(workspace, need, qzeros, z_bytes))
@@ -252,6 +259,12 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
         e = launch_tc(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
                       static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K, group_size,
                       zp_bias, static_cast<__half*>(out), workspace, c.tc, wp, st);
+        return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
+    }
+    if (c.gemv.mma) {
+        e = launch_gemv_mma(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
+                            static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K,
+                            group_size, zp_bias, static_cast<__half*>(out), workspace, c.gemv, wp, st);
         return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
     }
     if (gemv_smem_bytes(M, K, c.gemv.split_k) > 160 * 1024) return fail_arg("split_k too small for this K");
