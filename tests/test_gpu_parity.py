@@ -133,6 +133,14 @@ def test_odd_shapes(w, M, K, N, G, sym):
     assert_close(run(w, c), ref(c), f"odd {M}x{K}x{N} G{G}")
 
 
+@pytest.mark.parametrize("G", [16, 32, 48, 64, 80, 128, 192, 256])
+@pytest.mark.parametrize("M", [1, 3])
+def test_gemv_group_sizes(w, G, M):
+    # groups that are and are not multiples of the 64-row load unit; K spans several groups
+    c = synth.make_case(M, 8 * G, 384, G, sym=False, seed=G + M)
+    assert_close(run(w, c, kernel=w.KERNEL_GEMV), ref(c), f"GEMV G={G} M={M}")
+
+
 @pytest.mark.parametrize("split", [1, 2, 3, 7, 33, 256])
 def test_split_k_variants(w, split):
     c = synth.make_case(2, 2048, 1024, 128, sym=False, seed=21)
@@ -172,7 +180,7 @@ def test_repeatable_and_workspace_restored(w):
     o1 = run(w, c, workspace=ws)
     o2 = run(w, c, workspace=ws)
     assert torch.equal(o1, o2)
-    tiles = (c["N"] + 255) // 256
+    tiles = (c["N"] + 127) // 128                                # tiles are at least 128 columns wide
     assert int(ws[256:256 + 4 * tiles].count_nonzero()) == 0   # arrival counters back to zero
     assert w.w4a16_workspace_status(ws) == 0
 

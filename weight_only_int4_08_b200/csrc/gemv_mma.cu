@@ -1,6 +1,6 @@
-// Split-K GEMV for M <= 8 whose multiply-accumulate runs on warp-level tensor
-// instructions (mma.sync.m16n8k16, fp16 inputs, fp32 accumulation), with the
-// CUDA cores doing only the nibble unpack.
+// Stream-K GEMV for M <= 8 activation rows per launch, whose multiply-add runs
+// on warp-level tensor instructions (mma.sync.m16n8k16, fp16 inputs, fp32
+// accumulation) with the CUDA cores doing only the nibble unpack.
 //
 // Operation (vLLM PR #37352 analysis page, "코드 분석 1", `_w4a16_reference`):
 //   out[m, n] = fp16( sum_g s[g, n] * sum_{k in g} a[m, k] * (q[k, n] - z[g, n]) ),
@@ -8,23 +8,33 @@
 // fp16 activations are exact in the fp32 accumulator, and the group scale is
 // applied in fp32 to each group's accumulator.
 //
-// Why tensor instructions for a GEMV: measured on B200, the pure CUDA-core
-// inner loop (fp32 "magic number" unpack, packed FADD2/FFMA2) executes about
-// 41 instructions per packed word of 8 weights and is issue-bound well below
-// the HBM rate. Here a register holds two k-rows of four columns after one
-// ldmatrix.trans, and 9 instructions turn it into four exact (q - z) fp16 pairs
-// (0x6400 magic OR, fp16 subtract or fused scale-subtract); one mma.sync then
-// does 16 x 16 x 8 multiply-adds. The MMA's batch dimension (8) is padded for
-// M < 8; tensor throughput is not the bound.
+// Why tensor instructions for a GEMV: the pure CUDA-core inner loop (fp32
+// "magic number" unpack, packed FADD2/FFMA2) executes about 41 instructions per
+// packed word of 8 weights on B200 and is issue-bound below the HBM rate. Here
+// a register holds two k-rows of four columns after one ldmatrix.trans, and 9
+// instructions turn it into four exact (q - z) fp16 pairs (0x6400 magic OR,
+// fp16 subtract or fused scale-subtract); one mma.sync does 16 x 16 x 8
+// multiply-adds. The MMA's batch dimension (8) is padded for M < 8.
 //
-// Work decomposition: a CTA owns a 128-column tile (16 packed words per row)
-// and a K slab (split-K over gridDim.y); each of its 8 warps streams its own
-// run of 32-row blocks through a private ring of shared-memory stages filled
-// by 2-D TMA loads (64-byte swizzle, which makes the transposed ldmatrix reads
-// bank-conflict free). Swap-AB: the MMA's rows are output columns
-// (A = dequantised weights, transposed by ldmatrix), its columns the
-// activation rows (B). Warps are reduced through shared memory; split-K slabs
-// by the last-arriving CTA in slab order (deterministic).
+// Work decomposition (stream-K): the weight matrix is cut into units of one
+// 128-column tile x 64 rows (4 KB of packed weights), ordered tile by tile
+// along K. A single wave of resident CTAs takes equal contiguous runs of that
+// order, so every SM streams the same number of bytes whatever N and K are. A
+// CTA's run covers pieces ("fragments") of one to a few tiles; within a
+// fragment its 8 warps take equal runs of units, each through a private ring
+// of two shared-memory stages filled by 2-D TMA loads (weights with 64-byte
+// swizzle, which makes the transposed ldmatrix reads bank-conflict free, and
+// the activations of the same 64 rows) and tracked by one mbarrier per stage.
+// The stage shape follows a measurement on B200: streaming a 29 MB matrix,
+// TMA boxes of 64 B x 16..32 rows ran up to 2x slower than 4 KB boxes, and
+// about 128 KB in flight per SM was enough; more small boxes in flight made it
+// slower. Scales and zero words are copied one group ahead into a small
+// per-warp shared buffer (cp.async); each group's scaled sums are added to
+// fp32 totals kept in shared memory. At the end of a fragment the warps are
+// reduced in warp order; a tile covered by one CTA is
+// written directly, otherwise each CTA stores its fp32 partial in a slot of its
+// own and the last-arriving CTA sums the slots in CTA order (fixed order, no
+// floating-point atomics: bit-reproducible).
 //
 // Register layout (lane = 4 g + t): ldmatrix.trans gives thread (g, t) the
 // k-pair t of an 8-row matrix for columns 4g..4g+3 of a 32-column chunk; MMA 1
@@ -44,22 +54,46 @@ constexpr int kThreads = 256;
 constexpr int kWarps = 8;
 constexpr int kTileN = 128;
 constexpr int kTileWords = kTileN / 8;            // 16 packed words = 64 B per row
-constexpr int kRows = 32;                         // rows per TMA stage
-constexpr int kStage = kRows * kTileWords * 4;    // 2 KB
-constexpr int kRing = 4;                          // stages in flight per warp
-constexpr int kRingBytes = kWarps * kRing * kStage;
-constexpr int kMaxRowsPerCta = 2048;
+#ifndef W4A16_SK_ROWS
+#define W4A16_SK_ROWS 64
+#endif
+#ifndef W4A16_SK_RING
+#define W4A16_SK_RING 2
+#endif
+constexpr int kRows = W4A16_SK_ROWS;              // rows per unit / TMA stage (a multiple of 32)
+constexpr int kSteps = kRows / 16;                // 16-row MMA steps per stage
+constexpr int kWStage = kRows * kTileWords * 4;   // packed weight bytes per stage (4 KB)
+constexpr int kRing = W4A16_SK_RING;              // stages in flight per warp
+constexpr int kWRingBytes = kWarps * kRing * kWStage;
 
-struct MmaArgs {
-    const __half* a;      // [M, K]
+// Activation slot of one stage: MT rows x kRows fp16 (128 B per row). With more than four rows
+// the rows are loaded with 128-byte swizzle (so that ldmatrix reads of 8 rows hit 8 different
+// bank groups), which needs 1024-byte aligned slots; up to four rows the conflicts are cheaper
+// than the padding.
+__host__ __device__ constexpr bool a_swizzled(int mt) { return mt > 4; }
+__host__ __device__ constexpr int a_slot_bytes(int mt) { return a_swizzled(mt) ? 1024 : 2 * kRows * mt; }
+// Per warp, two group buffers: the tile's 128 scales (256 B) and 16 zero words (64 B).
+constexpr int kGrpBytes = 2 * kTileN + 4 * kTileWords;
+// Accumulator values per thread kept across groups: chunk c, entry i of the MMA accumulators
+// (only the even entries, batch 2t, matter for one activation row).
+__host__ __device__ constexpr int tot_per_chunk(int mt) { return mt > 1 ? 8 : 4; }
+// Dynamic shared memory: weight ring, activation ring, fp32 totals, group buffers, and the
+// warp-reduced sums of the (at most two) fragments shared with other CTAs.
+__host__ __device__ constexpr size_t sk_smem_bytes(int mt) {
+    return (size_t)kWRingBytes + (size_t)kWarps * kRing * a_slot_bytes(mt) +
+           (size_t)kWarps * 4 * tot_per_chunk(mt) * 32 * 4 + (size_t)kWarps * 2 * kGrpBytes + 2 * (size_t)mt * kTileN * 4;
+}
+
+struct SkArgs {
     const __half* s;      // [K/G, N]
     const uint32_t* z;    // [K/G, N/8] or nullptr
-    __half* out;          // [M, N] (row block)
-    float* partials;      // [split][MT][N]
-    uint32_t* counters;   // [col_tiles]
+    __half* out;          // [M, N] (this launch's row block)
+    float* partials;      // [tiles][slots][MT][128]
+    uint32_t* counters;   // [tiles]
     int* status;
-    int64_t N, K;
-    int G, zp_bias, split, s_vec, stall_loads;
+    int64_t N, K, units;  // units = tiles * nblk
+    int G, zp_bias, nblk, slots, stall_loads;
+    uint32_t magic;       // kMagic, passed at run time so that the and-or unpack compiles to one LOP3
     uint64_t wait_ns;
 };
 
@@ -73,7 +107,6 @@ __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
     return r;
 }
-
 __device__ __forceinline__ void mma16816(float& d0, float& d1, float& d2, float& d3, uint32_t a0, uint32_t a1,
                                          uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -82,266 +115,406 @@ __device__ __forceinline__ void mma16816(float& d0, float& d1, float& d2, float&
         : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Four 8x8 matrices, not transposed: thread t receives row t / 4, columns 2 (t % 4), 2 (t % 4) + 1.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(saddr)
+                 : "memory");
+}
+// Two transposed 8x8 matrices (rows given by threads 0..15).
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t saddr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(saddr)
+                 : "memory");
+}
 
-constexpr uint32_t kMagic = 0x64006400u;   // fp16 1024.0 in both halves
+constexpr uint32_t kMagic = 0x64006400u;      // fp16 1024.0 in both halves
+// Measured on B200: with both masks of (x & mask) | kMagic as compile-time constants the
+// compiler emits two logic instructions per unpacked register pair; with kMagic in a register
+// (a kernel argument) it emits one.
 constexpr uint32_t kSixteenth = 0x2C002C00u;  // fp16 1/16 in both halves
 
-// Per chunk (32 columns) and thread: four columns 4g..4g+3. Low-nibble columns
-// (j = 0, 2) subtract (1024 + z); high-nibble columns (j = 1, 3), unpacked as
-// 1024 + 16 q, are scaled by 1/16 and lose (64 + z) in one fused fp16 op.
-struct ChunkMeta {
-    uint32_t bias[4];   // j even: (1024 + z) x2; j odd: -(64 + z) x2  (fp16 bits)
-    float s[4];         // fp32 scales of the four columns
-};
+// CTA whose run of units contains unit u (runs are [floor(cU/C), floor((c+1)U/C))).
+__device__ __forceinline__ int64_t cta_of(int64_t u, int64_t U, int64_t C) { return ((u + 1) * C - 1) / U; }
 
+#ifndef W4A16_SK_MIN_CTAS
+#define W4A16_SK_MIN_CTAS 2
+#endif
 template <int MT>
-__global__ void __launch_bounds__(kThreads)
-gemv_mma_kernel(const __grid_constant__ CUtensorMap bmap, MmaArgs p) {
+__global__ void __launch_bounds__(kThreads, W4A16_SK_MIN_CTAS)
+gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap amap, SkArgs p) {
+    constexpr int kASlot = a_slot_bytes(MT);
     extern __shared__ __align__(1024) unsigned char s_dyn[];
-    unsigned char* ring = s_dyn;                                            // [8][kRing][2 KB]
-    uint32_t* s_act = reinterpret_cast<uint32_t*>(s_dyn + kRingBytes);      // [MT][rows/2] fp16 pairs
+    unsigned char* wring = s_dyn;                                        // [warp][kRing][kRows][64 B], 64-byte swizzle
+    unsigned char* aring = s_dyn + kWRingBytes;                          // [warp][kRing][MT][kRows] fp16
+    constexpr int NI = tot_per_chunk(MT);
+    // Per warp, the fragment's fp32 totals in thread-private order: [c * NI + i][lane].
+    float* tots = reinterpret_cast<float*>(aring + kWarps * kRing * kASlot);
     __shared__ __align__(8) uint64_t s_full[kWarps][kRing];
-    __shared__ int s_last;
+    __shared__ __align__(16) uint4 s_zero;   // the B rows past MT read these zeros
+    __shared__ int s_last[2];
     __shared__ volatile int s_abort;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float* tmine = tots + warp * 4 * NI * 32 + lane;
+    unsigned char* grp = reinterpret_cast<unsigned char*>(tots + kWarps * 4 * NI * 32) + warp * 2 * kGrpBytes;
+    float* keep = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(tots + kWarps * 4 * NI * 32) +
+                                           kWarps * 2 * kGrpBytes);   // [2][MT][128]
     const int g = lane >> 2, t = lane & 3;
     const int64_t nw = p.N / 8;
+    const int64_t U = p.units, C = gridDim.x, cta = blockIdx.x;
+    const int64_t u0 = U * cta / C, u1 = U * (cta + 1) / C;
+    const int64_t t0 = u0 / p.nblk;
+    const int nfrag = (int)((u1 - 1) / p.nblk - t0 + 1);
 
-    const int64_t nblk_total = (p.K + kRows - 1) / kRows;
-    const int64_t blk_begin = nblk_total * blockIdx.y / p.split;
-    const int64_t blk_end = nblk_total * (blockIdx.y + 1) / p.split;
-    const int64_t r_begin = blk_begin * kRows;
-    const int64_t r_end = min(blk_end * kRows, p.K);
-    const int rows_cta = (int)(r_end - r_begin);      // a multiple of 16
-    const int nblk = (int)(blk_end - blk_begin);
-    const int b_lo = nblk * warp / kWarps, b_hi = nblk * (warp + 1) / kWarps;
-    const int nmine = b_hi - b_lo;
+    // This warp's units of fragment f: k-blocks [lo, hi) of tile t0 + f.
+    auto frag_lo_hi = [&](int f, int& lo, int& hi) {
+        const int64_t tb = (t0 + f) * p.nblk;
+        const int64_t a = max(u0, tb) - tb, b = min(u1, tb + p.nblk) - tb;
+        lo = (int)(a + (b - a) * warp / kWarps);
+        hi = (int)(a + (b - a) * (warp + 1) / kWarps);
+    };
 
     if (threadIdx.x == 0) {
         s_abort = 0;
+        s_zero = make_uint4(0u, 0u, 0u, 0u);
         for (int w = 0; w < kWarps; ++w)
             for (int j = 0; j < kRing; ++j) ptx::mbar_init(ptx::smem_addr(&s_full[w][j]), 1);
         ptx::mbar_fence_init();
     }
     __syncthreads();
 
-    auto arm = [&](int j) {
-        const int slot = j % kRing;
+    // Load issue (lane 0): a cursor over this warp's units, one stage per unit.
+    int pf = 0, pkb = 0, phi = 0, armed = 0;
+    frag_lo_hi(0, pkb, phi);
+    auto arm_next = [&]() {
+        while (pkb >= phi) {
+            if (pf + 1 >= nfrag) return;
+            ++pf;
+            frag_lo_hi(pf, pkb, phi);
+        }
+        const int slot = armed % kRing;
         const uint32_t bar = ptx::smem_addr(&s_full[warp][slot]);
-        ptx::mbar_arrive_expect_tx(bar, (uint32_t)kStage);
-        ptx::tma_load_2d(ptx::smem_addr(ring + (size_t)(warp * kRing + slot) * kStage), &bmap,
-                         (int32_t)(blockIdx.x * kTileWords), (int32_t)(r_begin + (int64_t)(b_lo + j) * kRows), bar);
+        ptx::mbar_arrive_expect_tx(bar, (uint32_t)(kWStage + 2 * kRows * MT));
+        ptx::tma_load_2d(ptx::smem_addr(wring + (warp * kRing + slot) * kWStage), &bmap,
+                         (int32_t)((t0 + pf) * kTileWords), pkb * kRows, bar);
+        ptx::tma_load_2d(ptx::smem_addr(aring + (warp * kRing + slot) * kASlot), &amap, pkb * kRows, 0, bar);
+        ++pkb;
+        ++armed;
     };
     if (lane == 0 && !p.stall_loads) {
         ptx::prefetch_tensormap(&bmap);
-        for (int j = 0; j < min(kRing, nmine); ++j) arm(j);
+        ptx::prefetch_tensormap(&amap);
+        for (int j = 0; j < kRing; ++j) arm_next();
     }
-    // Activations of this slab as fp16 pairs (k, k+1).
-    const int half_rows = rows_cta / 2;
-    for (int i = threadIdx.x; i < MT * half_rows; i += kThreads) {
-        const int m = i / half_rows, r2 = i - m * half_rows;
-        s_act[i] = *reinterpret_cast<const uint32_t*>(p.a + (int64_t)m * p.K + r_begin + 2 * r2);
-    }
-    __syncthreads();
 
-    float tot[4][8], acc[4][8];
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) tot[c][i] = 0.f;
-    ChunkMeta meta[4];
-    int64_t g_cur = -1, g_next = 0;
-    const int64_t word0 = (int64_t)blockIdx.x * kTileWords + g / 2;   // + 4c: the word holding my columns
-    const int zshift = 16 * (g & 1);   // my first column is nibble 4 (g & 1) of that word
-    const int64_t ncol0 = (int64_t)blockIdx.x * kTileN + 4 * g;        // + 32c + j: my columns
-
-    auto group_end = [&]() {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            tot[c][0] = fmaf(meta[c].s[0], acc[c][0], tot[c][0]);
-            tot[c][1] = fmaf(meta[c].s[0], acc[c][1], tot[c][1]);
-            tot[c][2] = fmaf(meta[c].s[1], acc[c][2], tot[c][2]);
-            tot[c][3] = fmaf(meta[c].s[1], acc[c][3], tot[c][3]);
-            tot[c][4] = fmaf(meta[c].s[2], acc[c][4], tot[c][4]);
-            tot[c][5] = fmaf(meta[c].s[2], acc[c][5], tot[c][5]);
-            tot[c][6] = fmaf(meta[c].s[3], acc[c][6], tot[c][6]);
-            tot[c][7] = fmaf(meta[c].s[3], acc[c][7], tot[c][7]);
-        }
-    };
-    auto group_start = [&](int64_t gg) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int64_t word = word0 + 4 * c;
-            const bool ok = word < nw;
-            uint32_t zw = (uint32_t)p.zp_bias * 0x1111u;
-            if (p.z && ok) zw = __ldg(p.z + gg * nw + word) >> zshift;
-            meta[c].bias[0] = (0x6400u + (zw & 0xFu)) * 0x00010001u;
-            // -(64 + z): 0xD400 is -64 and one unit of the fraction is 1/16 there
-            meta[c].bias[1] = (0xD400u + 16u * ((zw >> 4) & 0xFu)) * 0x00010001u;
-            meta[c].bias[2] = (0x6400u + ((zw >> 8) & 0xFu)) * 0x00010001u;
-            meta[c].bias[3] = (0xD400u + 16u * ((zw >> 12) & 0xFu)) * 0x00010001u;
-            const __half* sp = p.s + gg * p.N + ncol0 + 32 * c;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) meta[c].s[j] = ok ? __half2float(__ldg(sp + j)) : 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[c][i] = 0.f;
-        }
-    };
-
+    const int zshift = 16 * (g & 1);       // my first column is nibble 4 (g & 1) of its zero word
+    const bool fast = (p.G % kRows) == 0;  // every unit lies in one group (and K % kRows == 0)
+    const int G = p.G;
     int consumed = 0;
-    for (int j = 0; j < nmine; ++j) {
-        const int slot = j % kRing;
-        const bool okw = ptx::mbar_wait(ptx::smem_addr(&s_full[warp][slot]), (uint32_t)((j / kRing) & 1), &s_abort,
-                                        p.wait_ns);
-        if (!__all_sync(0xffffffffu, okw)) break;
-        consumed = j + 1;
-        const int64_t rs = r_begin + (int64_t)(b_lo + j) * kRows;
-        const int64_t re = min(rs + kRows, r_end);
-        // Four chunks x four 8-row matrices, transposed: R[c][i] holds k-rows 8i + 2t, 8i + 2t + 1
-        // of columns 32c + 4g .. 32c + 4g + 3. My address row is `lane`; the 64-byte swizzle
-        // moves 16-byte chunk c of row r to chunk c ^ ((r >> 1) & 3).
-        const uint32_t sbase = ptx::smem_addr(ring + (size_t)(warp * kRing + slot) * kStage) + lane * 64;
-        uint32_t R[4][4];
+    bool failed = false;
+
+    uint32_t bias[4][4];  // j even: (1024 + z) x2; j odd: -(64 + z) x2 (fp16 bits)
+    auto set_bias = [&](int c, uint32_t zw) {
+        bias[c][0] = (0x6400u + (zw & 0xFu)) * 0x00010001u;
+        // -(64 + z): 0xD400 is -64 and one unit of the fraction is 1/16 there
+        bias[c][1] = (0xD400u + 16u * ((zw >> 4) & 0xFu)) * 0x00010001u;
+        bias[c][2] = (0x6400u + ((zw >> 8) & 0xFu)) * 0x00010001u;
+        bias[c][3] = (0xD400u + 16u * ((zw >> 12) & 0xFu)) * 0x00010001u;
+    };
+    if (!p.z) {  // one zero point for every column and group
 #pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::ldmatrix_x4_trans(sbase + 16 * (c ^ ((lane >> 1) & 3)), R[c]);
+        for (int c = 0; c < 4; ++c) set_bias(c, (uint32_t)p.zp_bias * 0x1111u);
+    }
+
+    for (int f = 0; f < nfrag; ++f) {
+        const int64_t tile = t0 + f;
+        int lo, hi;
+        frag_lo_hi(f, lo, hi);
+        const int64_t rend = min((int64_t)hi * kRows, p.K);
+        // This tile's scale row of group 0 (lane l copies scales 4l..4l+3) and zero row of group 0.
+        const __half* s_tile = p.s + tile * kTileN + 4 * lane;
+        const uint32_t* z_tile = p.z ? p.z + tile * kTileWords + lane : nullptr;
+        const bool s_ok = tile * kTileN + 32 * (lane / 8) < p.N;
+        const bool z_ok = p.z && lane < kTileWords && tile * kTileWords + lane < nw;
+
+        float acc[4][8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int64_t k0 = rs + 16 * h;
-            if (k0 >= re) break;
-            if (k0 >= g_next) {
-                if (g_cur >= 0) group_end();
-                g_cur = k0 / p.G;
-                g_next = (g_cur + 1) * p.G;
-                group_start(g_cur);
-            }
-            // B fragment: batch row g (zero past M), k-pairs t and t + 4 of this 16-k step.
-            uint32_t b0 = 0u, b1 = 0u;
-            if (g < MT) {
-                const uint32_t* ap = s_act + g * (rows_cta / 2) + (k0 - r_begin) / 2 + t;
-                b0 = ap[0];
-                b1 = ap[4];
-            }
+        for (int k = 0; k < 4 * NI; ++k) tmine[32 * k] = 0.f;
+
+        // Copy group gg's scales and zero words of this tile into group buffer gg & 1, one group
+        // ahead of use (lane l: scales 4l..4l+3; lanes 0..15: zero word l). Chunks past N get zeros.
+        auto load_group = [&](int64_t gg) {
+            unsigned char* gb = grp + (gg & 1) * kGrpBytes;
+            if (s_ok)
+                cp_async_8(ptx::smem_addr(gb + 8 * lane), s_tile + gg * p.N);
+            else
+                *reinterpret_cast<uint2*>(gb + 8 * lane) = make_uint2(0u, 0u);
+            if (z_ok) cp_async_4(ptx::smem_addr(gb + 2 * kTileN + 4 * lane), z_tile + gg * nw);
+            cp_async_commit();
+        };
+        // Groups advance one at a time: g_cur is the open group (from g_first), g_next its end row.
+        const int64_t g_first = (int64_t)lo * kRows / G;
+        int64_t g_cur = g_first - 1, g_next = g_first * G;
+        auto group_end = [&]() {
+            const unsigned char* gb = grp + (g_cur & 1) * kGrpBytes;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const uint32_t x0 = R[c][2 * h], x1 = R[c][2 * h + 1];
-                const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
-                const uint32_t e0a = hsub2((x0 & 0x000F000Fu) | kMagic, meta[c].bias[0]);
-                const uint32_t e1a = hfma2((x0 & 0x00F000F0u) | kMagic, kSixteenth, meta[c].bias[1]);
-                const uint32_t e0b = hsub2((x1 & 0x000F000Fu) | kMagic, meta[c].bias[0]);
-                const uint32_t e1b = hfma2((x1 & 0x00F000F0u) | kMagic, kSixteenth, meta[c].bias[1]);
-                const uint32_t e2a = hsub2((y0 & 0x000F000Fu) | kMagic, meta[c].bias[2]);
-                const uint32_t e3a = hfma2((y0 & 0x00F000F0u) | kMagic, kSixteenth, meta[c].bias[3]);
-                const uint32_t e2b = hsub2((y1 & 0x000F000Fu) | kMagic, meta[c].bias[2]);
-                const uint32_t e3b = hfma2((y1 & 0x00F000F0u) | kMagic, kSixteenth, meta[c].bias[3]);
+                const uint2 sc = *reinterpret_cast<const uint2*>(gb + 64 * c + 8 * g);
+                const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
+                const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
+                const float sj[4] = {s01.x, s01.y, s23.x, s23.y};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (MT > 1 || (i & 1) == 0) {
+                        float* tp = tmine + 32 * (c * NI + (MT > 1 ? i : i / 2));
+                        *tp = fmaf(sj[i >> 1], acc[c][i], *tp);
+                    }
+            }
+        };
+        // Start group gg (its buffer was filled one group earlier) and prefetch the next one.
+        auto group_start = [&](int64_t gg) {
+            cp_async_wait_all();
+            __syncwarp();   // every lane's copies have landed; every lane is done with the other buffer
+            const unsigned char* gb = grp + (gg & 1) * kGrpBytes;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (p.z) set_bias(c, *reinterpret_cast<const uint32_t*>(gb + 2 * kTileN + 4 * (4 * c + g / 2)) >> zshift);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[c][i] = 0.f;
+            }
+            if (g_next < rend) load_group(gg + 1);   // g_next is the first row of group gg + 1
+        };
+        // Dequantise two 8-row matrices of chunk c (k-rows r..r+7 in x0, r+8..r+15 in x1) and
+        // multiply them with the activation fragment (b0, b1).
+        const uint32_t magic = p.magic;
+        auto mma_chunk = [&](int c, uint32_t x0, uint32_t x1, uint32_t b0, uint32_t b1) {
+            {
+                const uint32_t e0a = hsub2((x0 & 0x000F000Fu) | magic, bias[c][0]);
+                const uint32_t e1a = hfma2((x0 & 0x00F000F0u) | magic, kSixteenth, bias[c][1]);
+                const uint32_t e0b = hsub2((x1 & 0x000F000Fu) | magic, bias[c][0]);
+                const uint32_t e1b = hfma2((x1 & 0x00F000F0u) | magic, kSixteenth, bias[c][1]);
                 mma16816(acc[c][0], acc[c][1], acc[c][2], acc[c][3], e0a, e1a, e0b, e1b, b0, b1);
+            }
+            {
+                const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
+                const uint32_t e2a = hsub2((y0 & 0x000F000Fu) | magic, bias[c][2]);
+                const uint32_t e3a = hfma2((y0 & 0x00F000F0u) | magic, kSixteenth, bias[c][3]);
+                const uint32_t e2b = hsub2((y1 & 0x000F000Fu) | magic, bias[c][2]);
+                const uint32_t e3b = hfma2((y1 & 0x00F000F0u) | magic, kSixteenth, bias[c][3]);
                 mma16816(acc[c][4], acc[c][5], acc[c][6], acc[c][7], e2a, e3a, e2b, e3b, b0, b1);
             }
-        }
-        // Every lane has consumed its ldmatrix results: the stage can be refilled.
-        __syncwarp();
-        if (lane == 0 && j + kRing < nmine && !p.stall_loads) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            arm(j + kRing);
-        }
-    }
-    if (g_cur >= 0) group_end();
+        };
 
-    if (s_abort) {
-        if (lane == 0) {
-            for (int j = consumed; j < min(nmine, consumed + kRing) && !p.stall_loads; ++j) {
-                volatile int dummy = 0;
-                ptx::mbar_wait(ptx::smem_addr(&s_full[warp][j % kRing]), (uint32_t)((j / kRing) & 1), &dummy, p.wait_ns);
+        if (lo < hi) load_group(g_first);
+        for (int kb = lo; kb < hi && !failed; ++kb) {
+            const int slot = consumed % kRing;
+            const bool okw = ptx::mbar_wait(ptx::smem_addr(&s_full[warp][slot]), (uint32_t)((consumed / kRing) & 1),
+                                            &s_abort, p.wait_ns);
+            if (!__all_sync(0xffffffffu, okw)) {
+                failed = true;
+                break;
             }
-            if (p.status) atomicExch(p.status, (int)W4A16_ERR_TIMEOUT);
+            ++consumed;
+            const int64_t rs = (int64_t)kb * kRows;
+            // Row r of the stage holds 16-byte chunk c at chunk c ^ ((r >> 1) & 3) (64-byte swizzle).
+            const uint32_t wst = ptx::smem_addr(wring + (warp * kRing + slot) * kWStage);
+            // B fragments (batch row g, k-pairs t and t + 4 of each 16-row step): one ldmatrix per two
+            // steps; lane i addresses row i % 8 (a zero row past MT) of the 8-k column block i / 8.
+            uint32_t bf[kSteps][2];
+#pragma unroll
+            for (int h2 = 0; h2 < kSteps / 2; ++h2) {
+                const int r = lane & 7, chunk = 4 * h2 + (lane >> 3);
+                const uint32_t addr = r < MT ? ptx::smem_addr(aring + (warp * kRing + slot) * kASlot) + r * 2 * kRows +
+                                                   16 * (a_swizzled(MT) ? (chunk ^ r) : chunk)
+                                             : ptx::smem_addr(&s_zero);
+                uint32_t B[4];
+                ldmatrix_x4(addr, B);
+                bf[2 * h2][0] = B[0];
+                bf[2 * h2][1] = B[1];
+                bf[2 * h2 + 1][0] = B[2];
+                bf[2 * h2 + 1][1] = B[3];
+            }
+            if (fast) {
+                if (rs >= g_next) {
+                    if (g_cur >= g_first) group_end();
+                    ++g_cur;
+                    g_next += G;
+                    group_start(g_cur);
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int q = 0; q < kRows / 32; ++q) {
+                        // rows 32q + lane; (32q + lane) >> 1 & 3 == lane >> 1 & 3
+                        uint32_t R[4];
+                        ptx::ldmatrix_x4_trans(wst + (32 * q + lane) * 64 + 16 * (c ^ ((lane >> 1) & 3)), R);
+                        mma_chunk(c, R[0], R[1], bf[2 * q][0], bf[2 * q][1]);
+                        mma_chunk(c, R[2], R[3], bf[2 * q + 1][0], bf[2 * q + 1][1]);
+                    }
+            } else {
+#pragma unroll
+                for (int h = 0; h < kSteps; ++h) {
+                    const int64_t k0 = rs + 16 * h;
+                    if (k0 >= rend) break;
+                    if (k0 >= g_next) {
+                        if (g_cur >= g_first) group_end();
+                        ++g_cur;
+                        g_next += G;
+                        group_start(g_cur);
+                    }
+                    const int row = 16 * h + (lane & 15);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t x0, x1;
+                        ldmatrix_x2_trans(wst + row * 64 + 16 * (c ^ ((row >> 1) & 3)), x0, x1);
+                        mma_chunk(c, x0, x1, bf[h][0], bf[h][1]);
+                    }
+                }
+            }
+            // Every lane has read the stage: it can be refilled.
+            __syncwarp();
+            if (lane == 0 && !p.stall_loads) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                arm_next();
+            }
         }
-    }
-    __syncthreads();  // rings are free: reuse them for the warp reduction
-    if (s_abort) return;
+        if (g_cur >= g_first && !failed) group_end();
 
-    // Warp reduction: s_red[w][m][128] (m < MT); thread values map to
-    // (column 32c + 4g + j, batch 2t + (i & 1)) with j = 0,1 from MMA 1 and 2,3 from MMA 2.
-    float* s_red = reinterpret_cast<float*>(s_dyn);
+        // ---- reduce fragment f over the warps (warp order) ----
+        // A tile held by this CTA alone is written out now; the first and the last fragment may be
+        // shared with neighbouring CTAs and are kept (keep[0], keep[1]) for the exchange at the end.
+        __syncthreads();
+        // s_abort is read by every thread between two barriers with no wait in between: uniform.
+        if (s_abort == 0) {
+            const bool shared_tile = cta_of(tile * p.nblk, U, C) != cta_of((tile + 1) * p.nblk - 1, U, C);
+            float* kp = keep + (f == 0 ? 0 : MT * kTileN);
+            for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
+                const int m = item / kTileN, nl = item % kTileN;
+                const int64_t n = tile * kTileN + nl;
+                // (m, nl) is entry i = 2 (nl % 4) + (m % 2) of chunk nl / 32 at lane 4 ((nl % 32) / 4) + m / 2
+                const int i = 2 * (nl & 3) + (m & 1);
+                const int src = 32 * ((nl >> 5) * NI + (MT > 1 ? i : i / 2)) + 4 * ((nl & 31) >> 2) + (m >> 1);
+                float v = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int m = 2 * t + (i & 1);
-            const int jcol = (i < 4) ? (i >> 1) : 2 + ((i - 4) >> 1);
-            if (m < MT) s_red[(warp * MT + m) * kTileN + 32 * c + 4 * g + jcol] = tot[c][i];
+                for (int w = 0; w < kWarps; ++w) v += tots[w * 4 * NI * 32 + src];
+                if (shared_tile) kp[item] = v;
+                else if (n < p.N) p.out[(int64_t)m * p.N + n] = __float2half_rn(v);
+            }
         }
-    __syncthreads();
-    const int64_t n0 = (int64_t)blockIdx.x * kTileN;
-    for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
-        const int m = item / kTileN, nl = item % kTileN;
-        float v = 0.f;
+        __syncthreads();  // the totals are free again
+    }
+
+    // ---- tiles shared with other CTAs: fp32 partials in CTA slots, summed by the last to arrive ----
+    if (s_abort == 0) {
+        int64_t d_tile[2];
+        int d_first[2], d_n[2];
+        bool d_on[2];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) v += s_red[(w * MT + m) * kTileN + nl];
-        const int64_t n = n0 + nl;
-        if (n < p.N) {
-            if (p.split == 1) p.out[(int64_t)m * p.N + n] = __float2half_rn(v);
-            else p.partials[((int64_t)blockIdx.y * MT + m) * p.N + n] = v;
+        for (int d = 0; d < 2; ++d) {
+            const int fd = d == 0 ? 0 : nfrag - 1;
+            d_tile[d] = t0 + fd;
+            const int64_t first = cta_of(d_tile[d] * p.nblk, U, C), last = cta_of((d_tile[d] + 1) * p.nblk - 1, U, C);
+            d_first[d] = (int)first;
+            d_n[d] = (int)(last - first + 1);
+            d_on[d] = d_n[d] > 1 && (d == 0 || nfrag > 1);
+            if (d_on[d]) {
+                float* slot_base = p.partials + ((d_tile[d] * p.slots + (cta - first)) * MT) * kTileN;
+                for (int item = threadIdx.x; item < MT * kTileN; item += kThreads)
+                    if (d_tile[d] * kTileN + item % kTileN < p.N) slot_base[item] = keep[d * MT * kTileN + item];
+            }
+        }
+        if (d_on[0] || d_on[1]) {
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+#pragma unroll
+                for (int d = 0; d < 2; ++d)
+                    s_last[d] = d_on[d] && atomicAdd(p.counters + d_tile[d], 1u) == (uint32_t)d_n[d] - 1;
+            }
+            __syncthreads();
+            if (s_last[0] || s_last[1]) {
+                __threadfence();
+#pragma unroll
+                for (int d = 0; d < 2; ++d) {
+                    if (!s_last[d]) continue;
+                    const float* tile_base = p.partials + (d_tile[d] * p.slots * MT) * kTileN;
+                    for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
+                        const int m = item / kTileN, nl = item % kTileN;
+                        const int64_t n = d_tile[d] * kTileN + nl;
+                        if (n >= p.N) continue;
+                        float v = 0.f;
+                        for (int y = 0; y < d_n[d]; ++y) v += __ldcg(tile_base + y * MT * kTileN + item);
+                        p.out[(int64_t)m * p.N + n] = __float2half_rn(v);
+                    }
+                    if (threadIdx.x == 0) p.counters[d_tile[d]] = 0u;
+                }
+            }
         }
     }
-    if (p.split == 1) return;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t ticket = atomicAdd(p.counters + blockIdx.x, 1u);
-        s_last = (ticket == (uint32_t)p.split - 1);
+
+    // A wait gave up: let the copies already issued land before the CTA's shared memory goes away.
+    cp_async_wait_all();
+    if (lane == 0 && consumed < armed) {
+        for (int j = consumed; j < armed; ++j) {
+            volatile int dummy = 0;
+            ptx::mbar_wait(ptx::smem_addr(&s_full[warp][j % kRing]), (uint32_t)((j / kRing) & 1), &dummy, p.wait_ns);
+        }
     }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
-        const int m = item / kTileN, nl = item % kTileN;
-        const int64_t n = n0 + nl;
-        if (n >= p.N) continue;
-        float v = 0.f;
-        for (int y = 0; y < p.split; ++y) v += __ldcg(p.partials + ((int64_t)y * MT + m) * p.N + n);
-        p.out[(int64_t)m * p.N + n] = __float2half_rn(v);
-    }
-    if (threadIdx.x == 0) p.counters[blockIdx.x] = 0u;
+    if (failed && lane == 0 && p.status) atomicExch(p.status, (int)W4A16_ERR_TIMEOUT);
 }
 
-using MmaFn = void (*)(CUtensorMap, MmaArgs);
+using SkFn = void (*)(CUtensorMap, CUtensorMap, SkArgs);
 
-MmaFn select_mma(int mt) {
+SkFn select_sk(int mt) {
     switch (mt) {
-        case 1: return gemv_mma_kernel<1>;
-        case 2: return gemv_mma_kernel<2>;
-        case 3: return gemv_mma_kernel<3>;
-        case 4: return gemv_mma_kernel<4>;
-        case 5: return gemv_mma_kernel<5>;
-        case 6: return gemv_mma_kernel<6>;
-        case 7: return gemv_mma_kernel<7>;
-        default: return gemv_mma_kernel<8>;
+        case 1: return gemv_sk_kernel<1>;
+        case 2: return gemv_sk_kernel<2>;
+        case 3: return gemv_sk_kernel<3>;
+        case 4: return gemv_sk_kernel<4>;
+        case 5: return gemv_sk_kernel<5>;
+        case 6: return gemv_sk_kernel<6>;
+        case 7: return gemv_sk_kernel<7>;
+        default: return gemv_sk_kernel<8>;
     }
 }
 
-std::atomic<int> g_mma_occ[9];
+std::atomic<int> g_sk_occ[9];
 
-size_t act_smem(int mt, int64_t rows) { return (size_t)mt * (size_t)rows * 2; }
-
-int mma_ctas_per_sm(int mt) {
-    int n = g_mma_occ[mt].load(std::memory_order_relaxed);
+// Resident CTAs per SM from the kernel's registers and shared memory.
+int sk_ctas_per_sm(int mt) {
+    int n = g_sk_occ[mt].load(std::memory_order_relaxed);
     if (n > 0) return n;
-    MmaFn k = select_mma(mt);
     cudaFuncAttributes fa{};
     int regs = 255;
-    if (cudaFuncGetAttributes(&fa, k) == cudaSuccess && fa.numRegs > 0) regs = fa.numRegs;
-    const size_t smem = kRingBytes + act_smem(mt, kMaxRowsPerCta) + fa.sharedSizeBytes + 1024;
+    size_t static_smem = 1024;
+    if (cudaFuncGetAttributes(&fa, select_sk(mt)) == cudaSuccess && fa.numRegs > 0) {
+        regs = fa.numRegs;
+        static_smem = fa.sharedSizeBytes;
+    }
+    const size_t smem = sk_smem_bytes(mt) + static_smem + 1024;   // + the per-CTA reservation
     const int by_smem = (int)((228 * 1024) / smem);
     const int by_regs = 65536 / (((regs + 7) / 8 * 8) * kThreads);
     n = std::max(1, std::min(by_smem, by_regs));
-    g_mma_occ[mt].store(n, std::memory_order_relaxed);
+    g_sk_occ[mt].store(n, std::memory_order_relaxed);
     return n;
 }
 
 }  // namespace
 
-bool gemv_mma_supported(int64_t N, const void* a, const void* b) {
-    return N % 32 == 0 && (reinterpret_cast<uintptr_t>(b) % 16) == 0 && (reinterpret_cast<uintptr_t>(a) % 4) == 0;
+bool gemv_mma_supported(int64_t N, const void* a, const void* b, const void* s) {
+    return N % 32 == 0 && (reinterpret_cast<uintptr_t>(b) % 16) == 0 && (reinterpret_cast<uintptr_t>(a) % 16) == 0 &&
+           (reinterpret_cast<uintptr_t>(s) % 8) == 0;
 }
 
 GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count) {
@@ -353,33 +526,25 @@ GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_r
     pl.m_rows = (int)std::min<int64_t>(M, 8);
     pl.col_tiles = (int)((N + kTileN - 1) / kTileN);
     const int64_t nblk = (K + kRows - 1) / kRows;
-    int64_t split;
+    const int64_t units = (int64_t)pl.col_tiles * nblk;
+    int64_t ctas;
     if (split_k_request > 0) {
-        split = std::min<int64_t>(split_k_request, nblk);
+        // As many CTAs as a split-K grid of that many slabs per tile would have.
+        ctas = (int64_t)split_k_request * pl.col_tiles;
     } else {
-        // Fill whole waves of resident CTAs best; count the fp32 partials a split writes and
-        // reads as traffic against the packed weights; at most kMaxRowsPerCta rows per CTA.
-        const int64_t slots = (int64_t)std::max(sm_count, 1) * mma_ctas_per_sm(pl.m_rows);
-        const int64_t smin = std::max<int64_t>(1, (K + kMaxRowsPerCta - 1) / kMaxRowsPerCta);
-        double best = -1.0;
-        split = smin;
-        for (int64_t sp = smin; sp <= std::min<int64_t>(nblk, 64); ++sp) {
-            const int64_t ctas = (int64_t)pl.col_tiles * sp;
-            const double waves = (double)((ctas + slots - 1) / slots);
-            const double fill = (double)ctas / (waves * (double)slots);
-            const double wb = (double)K * (double)N / 2;
-            const double pb = sp > 1 ? 2.0 * sp * pl.m_rows * (double)N * 4 : 0.0;
-            const double score = fill * wb / (wb + pb) / (1.0 + 0.02 * waves);
-            if (score > best + 1e-9) {
-                best = score;
-                split = sp;
-            }
-        }
+        // One wave of resident CTAs, each with at least a unit per warp on average.
+        ctas = std::min<int64_t>((int64_t)std::max(sm_count, 1) * sk_ctas_per_sm(pl.m_rows),
+                                 std::max<int64_t>(1, units / kWarps));
     }
-    pl.split_k = (int)std::max<int64_t>(1, split);
+    ctas = std::max<int64_t>(1, std::min(ctas, units));
+    pl.split_k = (int)ctas;  // the stream-K grid size
+    // A tile's units span at most ceil(nblk * C / U) + 1 CTAs.
+    pl.slots = (int)std::min<int64_t>(ctas, (nblk * ctas + units - 1) / units + 1);
     pl.counters_off = kWsHeader;
     pl.partials_off = align_up(kWsHeader + (size_t)pl.col_tiles * 4, 256);
-    pl.ws_bytes = pl.partials_off + (pl.split_k > 1 ? (size_t)pl.split_k * pl.m_rows * (size_t)N * 4 : 0);
+    // With exactly one CTA per tile no tile is shared and no partials are written.
+    const bool shared_tiles = ctas != pl.col_tiles;
+    pl.ws_bytes = shared_tiles ? pl.partials_off + (size_t)pl.col_tiles * pl.slots * pl.m_rows * kTileN * 4 : 0;
     return pl;
 }
 
@@ -387,39 +552,50 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
                             int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace,
                             const GemvPlan& pl, const WaitPolicy& wp, cudaStream_t st) {
     CUtensorMap bmap;
-    const cuuint64_t dims[2] = {(cuuint64_t)(N / 8), (cuuint64_t)K};
-    const cuuint64_t strides[1] = {(cuuint64_t)(N / 8) * 4};
-    const cuuint32_t box[2] = {(cuuint32_t)kTileWords, (cuuint32_t)kRows};
-    const cuuint32_t estr[2] = {1, 1};
-    cudaError_t e = encode_tensor_map(&bmap, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, (void*)b, dims, strides, box, estr,
-                                      CU_TENSOR_MAP_SWIZZLE_64B);
-    if (e != cudaSuccess) return e;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(N / 8), (cuuint64_t)K};
+        const cuuint64_t strides[1] = {(cuuint64_t)(N / 8) * 4};
+        const cuuint32_t box[2] = {(cuuint32_t)kTileWords, (cuuint32_t)kRows};
+        const cuuint32_t estr[2] = {1, 1};
+        cudaError_t e = encode_tensor_map(&bmap, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, (void*)b, dims, strides, box,
+                                          estr, CU_TENSOR_MAP_SWIZZLE_64B);
+        if (e != cudaSuccess) return e;
+    }
     const int64_t nblk = (K + kRows - 1) / kRows;
-    const int64_t rows_max = (nblk + pl.split_k - 1) / pl.split_k * kRows;
     char* ws = static_cast<char*>(workspace);
     for (int64_t m0 = 0; m0 < M; m0 += 8) {
         const int mt = (int)std::min<int64_t>(8, M - m0);
-        MmaArgs args;
-        args.a = a + m0 * K;
+        CUtensorMap amap;
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)mt};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)kRows, (cuuint32_t)mt};
+        const cuuint32_t estr[2] = {1, 1};
+        cudaError_t e = encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)(a + m0 * K), dims,
+                                          strides, box, estr,
+                                          a_swizzled(mt) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (e != cudaSuccess) return e;
+        SkArgs args;
         args.s = s;
         args.z = z;
         args.out = out + m0 * N;
         args.partials = reinterpret_cast<float*>(ws + pl.partials_off);
         args.counters = reinterpret_cast<uint32_t*>(ws + pl.counters_off);
-        args.status = reinterpret_cast<int*>(ws);
+        args.status = workspace ? reinterpret_cast<int*>(ws) : nullptr;
         args.N = N;
         args.K = K;
+        args.units = (int64_t)pl.col_tiles * nblk;
         args.G = G;
         args.zp_bias = zp_bias;
-        args.split = pl.split_k;
-        args.s_vec = 0;
+        args.nblk = (int)nblk;
+        args.slots = pl.slots;
+        args.magic = kMagic;
         args.stall_loads = wp.stall_loads;
         args.wait_ns = wp.limit_ns;
-        const size_t smem = kRingBytes + act_smem(mt, rows_max);
-        MmaFn k = select_mma(mt);
+        const size_t smem = sk_smem_bytes(mt);
+        SkFn k = select_sk(mt);
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        k<<<dim3((unsigned)pl.col_tiles, (unsigned)pl.split_k), kThreads, smem, st>>>(bmap, args);
+        k<<<dim3((unsigned)pl.split_k), kThreads, smem, st>>>(bmap, amap, args);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -90,8 +90,8 @@ w4a16_status w4a16_gemm_noalloc(const void* a, const void* b_packed, const void*
     // The array keeps the previous call's contents: the status word and the
     // arrival counters must start at zero, so clear them before every call.
     if (need > 0) {
-        // status word, then one counter per column tile (tiles are >= 256 columns wide)
-        const size_t header = std::min(need, kWsHeader + 4 * (size_t)(N / 256 + 2));
+        // status word, then one counter per column tile (tiles are at least 8 columns wide)
+        const size_t header = std::min(need, kWsHeader + 4 * (size_t)(N / 8 + 2));
         e = cudaMemsetAsync(scratch, 0, header, static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) {
             set_last_error(cudaGetErrorString(e));

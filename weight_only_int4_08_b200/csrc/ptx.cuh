@@ -59,11 +59,15 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // Wait for the phase of parity `parity` to complete. Gives up (returns false)
 // when *abort is set by another thread, or after `limit_ns` nanoseconds, in
 // which case it sets *abort itself.
+#ifndef W4A16_WAIT_SLEEP_NS
+#define W4A16_WAIT_SLEEP_NS 20000  // suspend hint of the polling try_wait (0: no hint)
+#endif
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (W4A16_WAIT_SLEEP_NS > 0 ? mbar_try_wait_sleep(bar, parity, W4A16_WAIT_SLEEP_NS) : mbar_try_wait(bar, parity))
+            return true;
         if (*abort) return false;
         if (globaltimer() - t0 > limit_ns) {
             *abort = 1;

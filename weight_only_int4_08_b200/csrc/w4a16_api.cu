@@ -86,7 +86,7 @@ struct Choice {
 // weights), the GEMV's 8-row blocks otherwise. Null pointers (workspace query)
 // count as aligned.
 Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms,
-              const void* a, const void* b) {
+              const void* a, const void* b, const void* s) {
     Choice c{};
     const int req = opts ? opts->kernel : W4A16_KERNEL_AUTO;
     const bool tc_ok = tc_supported(M, N, K, G, a ? a : (const void*)16, b ? b : (const void*)16);
@@ -96,7 +96,8 @@ Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_optio
     const int split = opts ? opts->split_k : 0;
     if (c.kernel == W4A16_KERNEL_TC) {
         if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, split);
-    } else if (req != W4A16_KERNEL_GEMV_FMA && gemv_mma_supported(N, a ? a : (const void*)16, b ? b : (const void*)16)) {
+    } else if (req != W4A16_KERNEL_GEMV_FMA &&
+               gemv_mma_supported(N, a ? a : (const void*)16, b ? b : (const void*)16, s ? s : (const void*)16)) {
         c.gemv = plan_gemv_mma(M, N, K, G, split, sms);
     } else {
         c.gemv = plan_gemv(M, N, K, G, split, sms, b ? max_vec_for(b) : 4, true);
@@ -233,7 +234,7 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
         set_error("unsupported: %s", "this library is built for sm_100 (B200) devices");
         return W4A16_ERR_UNSUPPORTED;
     }
-    Choice c = choose(M, N, K, group_size, opts, sms, a, b_packed);
+    Choice c = choose(M, N, K, group_size, opts, sms, a, b_packed, scales);
     if (c.kernel == W4A16_KERNEL_TC && !tc_supported(M, N, K, group_size, a, b_packed)) {
         set_error("unsupported: %s", "tensor-core kernel needs N % 128 == 0, K % 64 == 0, 16-byte aligned a and b_packed");
         return W4A16_ERR_UNSUPPORTED;
