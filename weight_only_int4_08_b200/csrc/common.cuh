@@ -31,7 +31,8 @@ struct GemvPlan {
     int m_rows;       // activation rows handled by one launch (1..8)
     int split_k;      // CTAs along K per column tile (stream-K GEMV: the grid size)
     int col_tiles;    // column tiles
-    int slots;        // stream-K GEMV: partial-sum slots per tile
+    int cluster;      // mma GEMV: CTAs per thread-block cluster
+    int cluster_tiles;  // mma GEMV: whole column tiles per cluster
     size_t ws_bytes;  // workspace bytes needed (0 when split_k == 1)
     size_t counters_off, partials_off;
 };
@@ -55,7 +56,7 @@ GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_reque
 
 // The stream-K mma.sync GEMV: N % 32 == 0, 16-byte aligned weights and activations,
 // 8-byte aligned scales.
-bool gemv_mma_supported(int64_t N, const void* a, const void* b, const void* s);
+bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s);
 GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count);
 cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M,
                             int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace,

@@ -65,6 +65,7 @@ constexpr int kSteps = kRows / 16;                // 16-row MMA steps per stage
 constexpr int kWStage = kRows * kTileWords * 4;   // packed weight bytes per stage (4 KB)
 constexpr int kRing = W4A16_SK_RING;              // stages in flight per warp
 constexpr int kWRingBytes = kWarps * kRing * kWStage;
+constexpr int kMaxCluster = 8;                    // portable thread-block cluster size
 
 // Activation slot of one stage: MT rows x kRows fp16 (128 B per row). With more than four rows
 // the rows are loaded with 128-byte swizzle (so that ldmatrix reads of 8 rows hit 8 different
@@ -88,11 +89,11 @@ struct SkArgs {
     const __half* s;      // [K/G, N]
     const uint32_t* z;    // [K/G, N/8] or nullptr
     __half* out;          // [M, N] (this launch's row block)
-    float* partials;      // [tiles][slots][MT][128]
-    uint32_t* counters;   // [tiles]
     int* status;
-    int64_t N, K, units;  // units = tiles * nblk
-    int G, zp_bias, nblk, slots, stall_loads;
+    int64_t N, K;
+    int tiles;            // 128-column tiles
+    int tiles_per_cluster;
+    int G, zp_bias, nblk, stall_loads;
     uint32_t magic;       // kMagic, passed at run time so that the and-or unpack compiles to one LOP3
     uint64_t wait_ns;
 };
@@ -144,45 +145,79 @@ constexpr uint32_t kMagic = 0x64006400u;      // fp16 1024.0 in both halves
 // (a kernel argument) it emits one.
 constexpr uint32_t kSixteenth = 0x2C002C00u;  // fp16 1/16 in both halves
 
-// CTA whose run of units contains unit u (runs are [floor(cU/C), floor((c+1)U/C))).
-__device__ __forceinline__ int64_t cta_of(int64_t u, int64_t U, int64_t C) { return ((u + 1) * C - 1) / U; }
+// Rank whose run of a cluster's units contains unit u (counted from the cluster's first unit);
+// runs are [floor(r U / S), floor((r + 1) U / S)).
+__device__ __forceinline__ int rank_of(int64_t u, int64_t U, int S) { return (int)(((u + 1) * S - 1) / U); }
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+// Shared-memory address of the same variable in CTA `rank` of the cluster, and a load from it.
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_cluster(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
 
 #ifndef W4A16_SK_MIN_CTAS
 #define W4A16_SK_MIN_CTAS 2
 #endif
-template <int MT>
+// FAST: the group size is a multiple of the 64-row unit, so a group starts only at a unit start
+// (and K is a multiple of 64); otherwise groups are tracked per 16-row step.
+template <int MT, bool FAST>
 __global__ void __launch_bounds__(kThreads, W4A16_SK_MIN_CTAS)
 gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap amap, SkArgs p) {
     constexpr int kASlot = a_slot_bytes(MT);
+    constexpr int NI = tot_per_chunk(MT);
     extern __shared__ __align__(1024) unsigned char s_dyn[];
     unsigned char* wring = s_dyn;                                        // [warp][kRing][kRows][64 B], 64-byte swizzle
     unsigned char* aring = s_dyn + kWRingBytes;                          // [warp][kRing][MT][kRows] fp16
-    constexpr int NI = tot_per_chunk(MT);
-    // Per warp, the fragment's fp32 totals in thread-private order: [c * NI + i][lane].
-    float* tots = reinterpret_cast<float*>(aring + kWarps * kRing * kASlot);
+    float* tots = reinterpret_cast<float*>(aring + kWarps * kRing * kASlot);  // [warp][c * NI + i][lane]
+    unsigned char* grps = reinterpret_cast<unsigned char*>(tots + kWarps * 4 * NI * 32);  // [warp][2][kGrpBytes]
+    float* keep = reinterpret_cast<float*>(grps + kWarps * 2 * kGrpBytes);                // [2][MT][128]
     __shared__ __align__(8) uint64_t s_full[kWarps][kRing];
     __shared__ __align__(16) uint4 s_zero;   // the B rows past MT read these zeros
-    __shared__ int s_last[2];
     __shared__ volatile int s_abort;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2;
     float* tmine = tots + warp * 4 * NI * 32 + lane;
-    unsigned char* grp = reinterpret_cast<unsigned char*>(tots + kWarps * 4 * NI * 32) + warp * 2 * kGrpBytes;
-    float* keep = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(tots + kWarps * 4 * NI * 32) +
-                                           kWarps * 2 * kGrpBytes);   // [2][MT][128]
-    const int g = lane >> 2, t = lane & 3;
-    const int64_t nw = p.N / 8;
-    const int64_t U = p.units, C = gridDim.x, cta = blockIdx.x;
-    const int64_t u0 = U * cta / C, u1 = U * (cta + 1) / C;
-    const int64_t t0 = u0 / p.nblk;
-    const int nfrag = (int)((u1 - 1) / p.nblk - t0 + 1);
+    unsigned char* grp = grps + warp * 2 * kGrpBytes;
+    const int nblk = p.nblk, G = p.G, K = (int)p.K;
+    const int nw = (int)(p.N / 8);
+    // My cluster owns tiles [tile_lo, tile_hi); its units (tile-major, 64-row blocks) are split in
+    // S equal contiguous runs, mine being run `rank`. Unit counts fit in 32 bits (the weights would
+    // not fit in memory otherwise; the host checks).
+    const int S = (int)cluster_nctarank(), rank = (int)cluster_ctarank();
+    const int tile_lo = (int)(blockIdx.x / S) * p.tiles_per_cluster;
+    const int tile_hi = min(tile_lo + p.tiles_per_cluster, p.tiles);
+    const int ubase = tile_lo * nblk, U = (tile_hi - tile_lo) * nblk;
+    const int u0 = ubase + (int)((int64_t)U * rank / S), u1 = ubase + (int)((int64_t)U * (rank + 1) / S);
+    const int t0 = u0 / nblk;
+    const int nfrag = u1 > u0 ? (u1 - 1) / nblk - t0 + 1 : 0;
 
     // This warp's units of fragment f: k-blocks [lo, hi) of tile t0 + f.
     auto frag_lo_hi = [&](int f, int& lo, int& hi) {
-        const int64_t tb = (t0 + f) * p.nblk;
-        const int64_t a = max(u0, tb) - tb, b = min(u1, tb + p.nblk) - tb;
-        lo = (int)(a + (b - a) * warp / kWarps);
-        hi = (int)(a + (b - a) * (warp + 1) / kWarps);
+        const int tb = (t0 + f) * nblk;
+        const int a = max(u0, tb) - tb, b = min(u1, tb + nblk) - tb;
+        lo = a + (b - a) * warp / kWarps;
+        hi = a + (b - a) * (warp + 1) / kWarps;
     };
 
     if (threadIdx.x == 0) {
@@ -194,6 +229,11 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     }
     __syncthreads();
 
+    // Per-warp shared-memory addresses of ring slot 0 (slot j adds j times the slot size).
+    const uint32_t bar0 = ptx::smem_addr(&s_full[warp][0]);
+    const uint32_t w0 = ptx::smem_addr(wring + warp * kRing * kWStage);
+    const uint32_t a0 = ptx::smem_addr(aring + warp * kRing * kASlot);
+
     // Load issue (lane 0): a cursor over this warp's units, one stage per unit.
     int pf = 0, pkb = 0, phi = 0, armed = 0;
     frag_lo_hi(0, pkb, phi);
@@ -204,11 +244,10 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             frag_lo_hi(pf, pkb, phi);
         }
         const int slot = armed % kRing;
-        const uint32_t bar = ptx::smem_addr(&s_full[warp][slot]);
+        const uint32_t bar = bar0 + 8 * slot;
         ptx::mbar_arrive_expect_tx(bar, (uint32_t)(kWStage + 2 * kRows * MT));
-        ptx::tma_load_2d(ptx::smem_addr(wring + (warp * kRing + slot) * kWStage), &bmap,
-                         (int32_t)((t0 + pf) * kTileWords), pkb * kRows, bar);
-        ptx::tma_load_2d(ptx::smem_addr(aring + (warp * kRing + slot) * kASlot), &amap, pkb * kRows, 0, bar);
+        ptx::tma_load_2d(w0 + slot * kWStage, &bmap, (t0 + pf) * kTileWords, pkb * kRows, bar);
+        ptx::tma_load_2d(a0 + slot * kASlot, &amap, pkb * kRows, 0, bar);
         ++pkb;
         ++armed;
     };
@@ -218,9 +257,8 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         for (int j = 0; j < kRing; ++j) arm_next();
     }
 
-    const int zshift = 16 * (g & 1);       // my first column is nibble 4 (g & 1) of its zero word
-    const bool fast = (p.G % kRows) == 0;  // every unit lies in one group (and K % kRows == 0)
-    const int G = p.G;
+    const int zshift = 16 * (g & 1);  // my first column is nibble 4 (g & 1) of its zero word
+    const uint32_t magic = p.magic;
     int consumed = 0;
     bool failed = false;
 
@@ -236,16 +274,27 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
         for (int c = 0; c < 4; ++c) set_bias(c, (uint32_t)p.zp_bias * 0x1111u);
     }
+    // B-fragment ldmatrix address of lane (row lane % 8, 8-k block lane / 8) in ring slot 0, or the
+    // zero row past MT; the second ldmatrix of a stage reads 4 blocks further.
+    const int br = lane & 7, bc = lane >> 3;
+    const uint32_t b_off = br < MT ? a0 + br * 2 * kRows : ptx::smem_addr(&s_zero);
+    const uint32_t b_col0 = br < MT ? 16 * (a_swizzled(MT) ? (bc ^ br) : bc) : 0;
+    const uint32_t b_col1 = br < MT ? 16 * (a_swizzled(MT) ? ((4 + bc) ^ br) : (4 + bc)) : 0;
+    const uint32_t b_slot = br < MT ? kASlot : 0;
+    // Weight ldmatrix.trans address of lane (row lane, 16-byte chunk c) under the 64-byte swizzle:
+    // row r holds chunk c at chunk c ^ ((r >> 1) & 3).
+    const uint32_t w_row = lane * 64;
+    const int w_sw = (lane >> 1) & 3;
 
     for (int f = 0; f < nfrag; ++f) {
-        const int64_t tile = t0 + f;
+        const int tile = t0 + f;
         int lo, hi;
         frag_lo_hi(f, lo, hi);
-        const int64_t rend = min((int64_t)hi * kRows, p.K);
-        // This tile's scale row of group 0 (lane l copies scales 4l..4l+3) and zero row of group 0.
-        const __half* s_tile = p.s + tile * kTileN + 4 * lane;
-        const uint32_t* z_tile = p.z ? p.z + tile * kTileWords + lane : nullptr;
-        const bool s_ok = tile * kTileN + 32 * (lane / 8) < p.N;
+        const int rend = min(hi * kRows, K);
+        // This tile's group-0 scale row (lane l copies scales 4l..4l+3) and zero row (lanes 0..15).
+        const __half* s_tile = p.s + (int64_t)tile * kTileN + 4 * lane;
+        const uint32_t* z_tile = p.z ? p.z + (int64_t)tile * kTileWords + lane : nullptr;
+        const bool s_ok = (int64_t)tile * kTileN + 32 * (lane / 8) < p.N;
         const bool z_ok = p.z && lane < kTileWords && tile * kTileWords + lane < nw;
 
         float acc[4][8];
@@ -253,19 +302,19 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         for (int k = 0; k < 4 * NI; ++k) tmine[32 * k] = 0.f;
 
         // Copy group gg's scales and zero words of this tile into group buffer gg & 1, one group
-        // ahead of use (lane l: scales 4l..4l+3; lanes 0..15: zero word l). Chunks past N get zeros.
-        auto load_group = [&](int64_t gg) {
+        // ahead of use. Chunks past N get zero scales.
+        auto load_group = [&](int gg) {
             unsigned char* gb = grp + (gg & 1) * kGrpBytes;
             if (s_ok)
-                cp_async_8(ptx::smem_addr(gb + 8 * lane), s_tile + gg * p.N);
+                cp_async_8(ptx::smem_addr(gb + 8 * lane), s_tile + (int64_t)gg * p.N);
             else
                 *reinterpret_cast<uint2*>(gb + 8 * lane) = make_uint2(0u, 0u);
-            if (z_ok) cp_async_4(ptx::smem_addr(gb + 2 * kTileN + 4 * lane), z_tile + gg * nw);
+            if (z_ok) cp_async_4(ptx::smem_addr(gb + 2 * kTileN + 4 * lane), z_tile + (int64_t)gg * nw);
             cp_async_commit();
         };
         // Groups advance one at a time: g_cur is the open group (from g_first), g_next its end row.
-        const int64_t g_first = (int64_t)lo * kRows / G;
-        int64_t g_cur = g_first - 1, g_next = g_first * G;
+        const int g_first = lo * kRows / G;
+        int g_cur = g_first - 1, g_next = g_first * G;
         auto group_end = [&]() {
             const unsigned char* gb = grp + (g_cur & 1) * kGrpBytes;
 #pragma unroll
@@ -283,7 +332,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             }
         };
         // Start group gg (its buffer was filled one group earlier) and prefetch the next one.
-        auto group_start = [&](int64_t gg) {
+        auto group_start = [&](int gg) {
             cp_async_wait_all();
             __syncwarp();   // every lane's copies have landed; every lane is done with the other buffer
             const unsigned char* gb = grp + (gg & 1) * kGrpBytes;
@@ -295,9 +344,14 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             }
             if (g_next < rend) load_group(gg + 1);   // g_next is the first row of group gg + 1
         };
+        auto advance_group = [&]() {
+            if (g_cur >= g_first) group_end();
+            ++g_cur;
+            g_next += G;
+            group_start(g_cur);
+        };
         // Dequantise two 8-row matrices of chunk c (k-rows r..r+7 in x0, r+8..r+15 in x1) and
         // multiply them with the activation fragment (b0, b1).
-        const uint32_t magic = p.magic;
         auto mma_chunk = [&](int c, uint32_t x0, uint32_t x1, uint32_t b0, uint32_t b1) {
             {
                 const uint32_t e0a = hsub2((x0 & 0x000F000Fu) | magic, bias[c][0]);
@@ -319,60 +373,47 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         if (lo < hi) load_group(g_first);
         for (int kb = lo; kb < hi && !failed; ++kb) {
             const int slot = consumed % kRing;
-            const bool okw = ptx::mbar_wait(ptx::smem_addr(&s_full[warp][slot]), (uint32_t)((consumed / kRing) & 1),
-                                            &s_abort, p.wait_ns);
+            const bool okw = ptx::mbar_wait(bar0 + 8 * slot, (uint32_t)((consumed / kRing) & 1), &s_abort, p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) {
                 failed = true;
                 break;
             }
             ++consumed;
-            const int64_t rs = (int64_t)kb * kRows;
-            // Row r of the stage holds 16-byte chunk c at chunk c ^ ((r >> 1) & 3) (64-byte swizzle).
-            const uint32_t wst = ptx::smem_addr(wring + (warp * kRing + slot) * kWStage);
-            // B fragments (batch row g, k-pairs t and t + 4 of each 16-row step): one ldmatrix per two
-            // steps; lane i addresses row i % 8 (a zero row past MT) of the 8-k column block i / 8.
+            const int rs = kb * kRows;
+            const uint32_t wst = w0 + slot * kWStage;
+            // B fragments (batch row g, k-pairs t and t + 4 of each 16-row step), two steps per ldmatrix.
             uint32_t bf[kSteps][2];
-#pragma unroll
-            for (int h2 = 0; h2 < kSteps / 2; ++h2) {
-                const int r = lane & 7, chunk = 4 * h2 + (lane >> 3);
-                const uint32_t addr = r < MT ? ptx::smem_addr(aring + (warp * kRing + slot) * kASlot) + r * 2 * kRows +
-                                                   16 * (a_swizzled(MT) ? (chunk ^ r) : chunk)
-                                             : ptx::smem_addr(&s_zero);
+            {
                 uint32_t B[4];
-                ldmatrix_x4(addr, B);
-                bf[2 * h2][0] = B[0];
-                bf[2 * h2][1] = B[1];
-                bf[2 * h2 + 1][0] = B[2];
-                bf[2 * h2 + 1][1] = B[3];
+                ldmatrix_x4(b_off + slot * b_slot + b_col0, B);
+                bf[0][0] = B[0];
+                bf[0][1] = B[1];
+                bf[1][0] = B[2];
+                bf[1][1] = B[3];
+                ldmatrix_x4(b_off + slot * b_slot + b_col1, B);
+                bf[2][0] = B[0];
+                bf[2][1] = B[1];
+                bf[3][0] = B[2];
+                bf[3][1] = B[3];
             }
-            if (fast) {
-                if (rs >= g_next) {
-                    if (g_cur >= g_first) group_end();
-                    ++g_cur;
-                    g_next += G;
-                    group_start(g_cur);
-                }
+            if constexpr (FAST) {
+                if (rs >= g_next) advance_group();
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int q = 0; q < kRows / 32; ++q) {
-                        // rows 32q + lane; (32q + lane) >> 1 & 3 == lane >> 1 & 3
+                        // rows 32q + lane; ((32q + lane) >> 1) & 3 == (lane >> 1) & 3
                         uint32_t R[4];
-                        ptx::ldmatrix_x4_trans(wst + (32 * q + lane) * 64 + 16 * (c ^ ((lane >> 1) & 3)), R);
+                        ptx::ldmatrix_x4_trans(wst + 32 * q * 64 + w_row + 16 * (c ^ w_sw), R);
                         mma_chunk(c, R[0], R[1], bf[2 * q][0], bf[2 * q][1]);
                         mma_chunk(c, R[2], R[3], bf[2 * q + 1][0], bf[2 * q + 1][1]);
                     }
             } else {
 #pragma unroll
                 for (int h = 0; h < kSteps; ++h) {
-                    const int64_t k0 = rs + 16 * h;
+                    const int k0 = rs + 16 * h;
                     if (k0 >= rend) break;
-                    if (k0 >= g_next) {
-                        if (g_cur >= g_first) group_end();
-                        ++g_cur;
-                        g_next += G;
-                        group_start(g_cur);
-                    }
+                    if (k0 >= g_next) advance_group();
                     const int row = 16 * h + (lane & 15);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
@@ -393,15 +434,15 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 
         // ---- reduce fragment f over the warps (warp order) ----
         // A tile held by this CTA alone is written out now; the first and the last fragment may be
-        // shared with neighbouring CTAs and are kept (keep[0], keep[1]) for the exchange at the end.
+        // shared with other CTAs of the cluster and are kept (keep[0], keep[1]) for the exchange.
         __syncthreads();
         // s_abort is read by every thread between two barriers with no wait in between: uniform.
         if (s_abort == 0) {
-            const bool shared_tile = cta_of(tile * p.nblk, U, C) != cta_of((tile + 1) * p.nblk - 1, U, C);
+            const bool shared_tile = rank_of(tile * nblk - ubase, U, S) != rank_of((tile + 1) * nblk - 1 - ubase, U, S);
             float* kp = keep + (f == 0 ? 0 : MT * kTileN);
             for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
                 const int m = item / kTileN, nl = item % kTileN;
-                const int64_t n = tile * kTileN + nl;
+                const int64_t n = (int64_t)tile * kTileN + nl;
                 // (m, nl) is entry i = 2 (nl % 4) + (m % 2) of chunk nl / 32 at lane 4 ((nl % 32) / 4) + m / 2
                 const int i = 2 * (nl & 3) + (m & 1);
                 const int src = 32 * ((nl >> 5) * NI + (MT > 1 ? i : i / 2)) + 4 * ((nl & 31) >> 2) + (m >> 1);
@@ -415,60 +456,39 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         __syncthreads();  // the totals are free again
     }
 
-    // ---- tiles shared with other CTAs: fp32 partials in CTA slots, summed by the last to arrive ----
+    // ---- tiles shared within the cluster: the first CTA touching a tile sums every part, in rank
+    // order, from the CTAs' shared memory (distributed shared memory), then writes the tile ----
+    cluster_sync();
     if (s_abort == 0) {
-        int64_t d_tile[2];
-        int d_first[2], d_n[2];
-        bool d_on[2];
 #pragma unroll
         for (int d = 0; d < 2; ++d) {
-            const int fd = d == 0 ? 0 : nfrag - 1;
-            d_tile[d] = t0 + fd;
-            const int64_t first = cta_of(d_tile[d] * p.nblk, U, C), last = cta_of((d_tile[d] + 1) * p.nblk - 1, U, C);
-            d_first[d] = (int)first;
-            d_n[d] = (int)(last - first + 1);
-            d_on[d] = d_n[d] > 1 && (d == 0 || nfrag > 1);
-            if (d_on[d]) {
-                float* slot_base = p.partials + ((d_tile[d] * p.slots + (cta - first)) * MT) * kTileN;
-                for (int item = threadIdx.x; item < MT * kTileN; item += kThreads)
-                    if (d_tile[d] * kTileN + item % kTileN < p.N) slot_base[item] = keep[d * MT * kTileN + item];
+            if (d >= nfrag || (d == 1 && nfrag == 1)) continue;
+            const int tile = t0 + (d == 0 ? 0 : nfrag - 1);
+            const int first = rank_of(tile * nblk - ubase, U, S), last = rank_of((tile + 1) * nblk - 1 - ubase, U, S);
+            if (first == last || first != rank) continue;
+            uint32_t src[kMaxCluster];   // keep slot of this tile in each contributing CTA (first tile of its run: 0)
+            for (int rr = first; rr <= last; ++rr) {
+                const int first_tile_rr = (ubase + (int)((int64_t)U * rr / S)) / nblk;
+                src[rr - first] = map_rank(ptx::smem_addr(keep + (tile == first_tile_rr ? 0 : MT * kTileN)), (uint32_t)rr);
             }
-        }
-        if (d_on[0] || d_on[1]) {
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) {
-#pragma unroll
-                for (int d = 0; d < 2; ++d)
-                    s_last[d] = d_on[d] && atomicAdd(p.counters + d_tile[d], 1u) == (uint32_t)d_n[d] - 1;
-            }
-            __syncthreads();
-            if (s_last[0] || s_last[1]) {
-                __threadfence();
-#pragma unroll
-                for (int d = 0; d < 2; ++d) {
-                    if (!s_last[d]) continue;
-                    const float* tile_base = p.partials + (d_tile[d] * p.slots * MT) * kTileN;
-                    for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
-                        const int m = item / kTileN, nl = item % kTileN;
-                        const int64_t n = d_tile[d] * kTileN + nl;
-                        if (n >= p.N) continue;
-                        float v = 0.f;
-                        for (int y = 0; y < d_n[d]; ++y) v += __ldcg(tile_base + y * MT * kTileN + item);
-                        p.out[(int64_t)m * p.N + n] = __float2half_rn(v);
-                    }
-                    if (threadIdx.x == 0) p.counters[d_tile[d]] = 0u;
-                }
+            for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
+                const int m = item / kTileN, nl = item % kTileN;
+                const int64_t n = (int64_t)tile * kTileN + nl;
+                if (n >= p.N) continue;
+                float v = 0.f;
+                for (int rr = first; rr <= last; ++rr) v += ld_cluster(src[rr - first] + 4 * item);
+                p.out[(int64_t)m * p.N + n] = __float2half_rn(v);
             }
         }
     }
+    cluster_sync();   // no CTA leaves while another still reads its shared memory
 
     // A wait gave up: let the copies already issued land before the CTA's shared memory goes away.
     cp_async_wait_all();
     if (lane == 0 && consumed < armed) {
         for (int j = consumed; j < armed; ++j) {
             volatile int dummy = 0;
-            ptx::mbar_wait(ptx::smem_addr(&s_full[warp][j % kRing]), (uint32_t)((j / kRing) & 1), &dummy, p.wait_ns);
+            ptx::mbar_wait(bar0 + 8 * (j % kRing), (uint32_t)((j / kRing) & 1), &dummy, p.wait_ns);
         }
     }
     if (failed && lane == 0 && p.status) atomicExch(p.status, (int)W4A16_ERR_TIMEOUT);
@@ -476,18 +496,21 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 
 using SkFn = void (*)(CUtensorMap, CUtensorMap, SkArgs);
 
-SkFn select_sk(int mt) {
+template <bool FAST>
+SkFn select_sk_t(int mt) {
     switch (mt) {
-        case 1: return gemv_sk_kernel<1>;
-        case 2: return gemv_sk_kernel<2>;
-        case 3: return gemv_sk_kernel<3>;
-        case 4: return gemv_sk_kernel<4>;
-        case 5: return gemv_sk_kernel<5>;
-        case 6: return gemv_sk_kernel<6>;
-        case 7: return gemv_sk_kernel<7>;
-        default: return gemv_sk_kernel<8>;
+        case 1: return gemv_sk_kernel<1, FAST>;
+        case 2: return gemv_sk_kernel<2, FAST>;
+        case 3: return gemv_sk_kernel<3, FAST>;
+        case 4: return gemv_sk_kernel<4, FAST>;
+        case 5: return gemv_sk_kernel<5, FAST>;
+        case 6: return gemv_sk_kernel<6, FAST>;
+        case 7: return gemv_sk_kernel<7, FAST>;
+        default: return gemv_sk_kernel<8, FAST>;
     }
 }
+// Occupancy queries use the FAST instance (both have the same shared memory and launch bounds).
+SkFn select_sk(int mt, bool fast = true) { return fast ? select_sk_t<true>(mt) : select_sk_t<false>(mt); }
 
 std::atomic<int> g_sk_occ[9];
 
@@ -510,11 +533,42 @@ int sk_ctas_per_sm(int mt) {
     return n;
 }
 
+std::atomic<int> g_sk_clusters[9][kMaxCluster + 1];
+
+// Clusters of S CTAs that can be resident at once (clusters are placed within one GPC each, so
+// this can be less than the resident CTAs divided by S).
+int sk_max_clusters(int mt, int S) {
+    int n = g_sk_clusters[mt][S].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    SkFn k = select_sk(mt);
+    const size_t smem = sk_smem_bytes(mt);
+    n = 0;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)S);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)S;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, k, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();  // a failed query must not leak into the next launch check
+    if (n <= 0) n = 1;
+    g_sk_clusters[mt][S].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 }  // namespace
 
-bool gemv_mma_supported(int64_t N, const void* a, const void* b, const void* s) {
-    return N % 32 == 0 && (reinterpret_cast<uintptr_t>(b) % 16) == 0 && (reinterpret_cast<uintptr_t>(a) % 16) == 0 &&
-           (reinterpret_cast<uintptr_t>(s) % 8) == 0;
+bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s) {
+    const int64_t units = (N + kTileN - 1) / kTileN * ((K + kRows - 1) / kRows);   // counted in 32 bits
+    return N % 32 == 0 && units < ((int64_t)1 << 31) && (reinterpret_cast<uintptr_t>(b) % 16) == 0 &&
+           (reinterpret_cast<uintptr_t>(a) % 16) == 0 && (reinterpret_cast<uintptr_t>(s) % 8) == 0;
 }
 
 GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count) {
@@ -525,26 +579,37 @@ GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_r
     pl.vec = 1;
     pl.m_rows = (int)std::min<int64_t>(M, 8);
     pl.col_tiles = (int)((N + kTileN - 1) / kTileN);
-    const int64_t nblk = (K + kRows - 1) / kRows;
-    const int64_t units = (int64_t)pl.col_tiles * nblk;
-    int64_t ctas;
+    const int64_t T = pl.col_tiles, nblk = (K + kRows - 1) / kRows;
+    int best_s = 1, best_k = 1;
     if (split_k_request > 0) {
-        // As many CTAs as a split-K grid of that many slabs per tile would have.
-        ctas = (int64_t)split_k_request * pl.col_tiles;
+        // That many CTAs per tile (at most a cluster, at most one per unit).
+        best_s = (int)std::min<int64_t>(std::min(split_k_request, kMaxCluster), nblk);
     } else {
-        // One wave of resident CTAs, each with at least a unit per warp on average.
-        ctas = std::min<int64_t>((int64_t)std::max(sm_count, 1) * sk_ctas_per_sm(pl.m_rows),
-                                 std::max<int64_t>(1, units / kWarps));
+        // Clusters of S CTAs over k whole tiles each, all resident at once: the fewest units per
+        // CTA wins, then the most CTAs.
+        const int64_t slots = (int64_t)std::max(sm_count, 1) * sk_ctas_per_sm(pl.m_rows);
+        int64_t best_cost = INT64_MAX, best_ctas = 0;
+        for (int S = 1; S <= kMaxCluster; ++S) {
+            const int64_t qmax = std::min<int64_t>({T, slots / S, (int64_t)sk_max_clusters(pl.m_rows, S)});
+            for (int64_t Q = 1; Q <= qmax; ++Q) {
+                const int64_t k = (T + Q - 1) / Q;
+                if ((Q - 1) * k >= T) continue;   // the same k with fewer clusters
+                const int64_t ctas = Q * S;
+                if (S > nblk) continue;   // every CTA of every cluster (the last one may be short) gets a unit
+                const int64_t cost = (k * nblk + S - 1) / S;
+                if (cost < best_cost || (cost == best_cost && ctas > best_ctas)) {
+                    best_cost = cost;
+                    best_ctas = ctas;
+                    best_s = S;
+                    best_k = (int)k;
+                }
+            }
+        }
     }
-    ctas = std::max<int64_t>(1, std::min(ctas, units));
-    pl.split_k = (int)ctas;  // the stream-K grid size
-    // A tile's units span at most ceil(nblk * C / U) + 1 CTAs.
-    pl.slots = (int)std::min<int64_t>(ctas, (nblk * ctas + units - 1) / units + 1);
-    pl.counters_off = kWsHeader;
-    pl.partials_off = align_up(kWsHeader + (size_t)pl.col_tiles * 4, 256);
-    // With exactly one CTA per tile no tile is shared and no partials are written.
-    const bool shared_tiles = ctas != pl.col_tiles;
-    pl.ws_bytes = shared_tiles ? pl.partials_off + (size_t)pl.col_tiles * pl.slots * pl.m_rows * kTileN * 4 : 0;
+    pl.cluster = best_s;
+    pl.cluster_tiles = best_k;
+    pl.split_k = (int)((T + best_k - 1) / best_k) * best_s;  // the grid size
+    pl.ws_bytes = 0;  // partial sums stay in the clusters' shared memory
     return pl;
 }
 
@@ -578,25 +643,34 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         args.s = s;
         args.z = z;
         args.out = out + m0 * N;
-        args.partials = reinterpret_cast<float*>(ws + pl.partials_off);
-        args.counters = reinterpret_cast<uint32_t*>(ws + pl.counters_off);
         args.status = workspace ? reinterpret_cast<int*>(ws) : nullptr;
         args.N = N;
         args.K = K;
-        args.units = (int64_t)pl.col_tiles * nblk;
+        args.tiles = pl.col_tiles;
+        args.tiles_per_cluster = pl.cluster_tiles;
         args.G = G;
         args.zp_bias = zp_bias;
         args.nblk = (int)nblk;
-        args.slots = pl.slots;
         args.magic = kMagic;
         args.stall_loads = wp.stall_loads;
         args.wait_ns = wp.limit_ns;
         const size_t smem = sk_smem_bytes(mt);
-        SkFn k = select_sk(mt);
+        SkFn k = select_sk(mt, G % kRows == 0);
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        k<<<dim3((unsigned)pl.split_k), kThreads, smem, st>>>(bmap, amap, args);
-        e = cudaGetLastError();
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)pl.split_k);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)pl.cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, k, bmap, amap, args);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -97,7 +97,7 @@ Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_optio
     if (c.kernel == W4A16_KERNEL_TC) {
         if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, split);
     } else if (req != W4A16_KERNEL_GEMV_FMA &&
-               gemv_mma_supported(N, a ? a : (const void*)16, b ? b : (const void*)16, s ? s : (const void*)16)) {
+               gemv_mma_supported(N, K, a ? a : (const void*)16, b ? b : (const void*)16, s ? s : (const void*)16)) {
         c.gemv = plan_gemv_mma(M, N, K, G, split, sms);
     } else {
         c.gemv = plan_gemv(M, N, K, G, split, sms, b ? max_vec_for(b) : 4, true);
@@ -239,14 +239,14 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
         set_error("unsupported: %s", "tensor-core kernel needs N % 128 == 0, K % 64 == 0, 16-byte aligned a and b_packed");
         return W4A16_ERR_UNSUPPORTED;
     }
-    const size_t need = c.kernel == W4A16_KERNEL_TC ? c.tc.ws_bytes : c.gemv.ws_bytes;
+    // The documented contract: a workspace of at least what the size query advertises for these
+    // arguments (a bound over the kernels the automatic choice may take), whatever this call uses.
+    const size_t need = std::max(c.kernel == W4A16_KERNEL_TC ? c.tc.ws_bytes : c.gemv.ws_bytes,
+                                 ws_bound(M, N, K, group_size, opts, sms));
     if (need > 0) {
         if (!workspace) return fail_arg("workspace required (see w4a16_gemm_workspace_bytes)");
         if (!aligned(workspace, 256)) return fail_arg("workspace must be 256-byte aligned");
-        // The documented contract: at least what the size query advertises for these arguments
-        // (a bound over the kernels the automatic choice may take), not just what this plan uses.
-        if (workspace_bytes < std::max(need, ws_bound(M, N, K, group_size, opts, sms)))
-            return fail_arg("workspace too small");
+        if (workspace_bytes < need) return fail_arg("workspace too small");
         if (overlaps(workspace, need, out, o_bytes) || overlaps(workspace, need, a, a_bytes) ||
             overlaps(workspace, need, b_packed, b_bytes) || overlaps(workspace, need, scales, s_bytes) ||
             overlaps(workspace, need, qzeros, z_bytes))
