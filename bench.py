@@ -211,10 +211,10 @@ def measure_problem(torch, prob, steps_per_graph, reps):
 def summary(prob, per_step_s, peaks, tensor_bound):
     gbs = prob.bytes / per_step_s / 1e9
     tfs = prob.flops / per_step_s / 1e12
+    # every path multiplies on the tensor cores (mma.sync for M <= 8, tcgen05 above)
     t_hbm = prob.bytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = prob.flops / (peaks["bf16_tflops"] * 1e12)
-    t_fp32 = prob.flops / (148 * 128 * 2 * 1.965e9)
-    t_roof = max(t_hbm, t_tc if tensor_bound else t_fp32)
+    t_roof = max(t_hbm, t_tc)
     return {"us": round(per_step_s * 1e6, 3), "GB/s": round(gbs, 1), "TFLOP/s": round(tfs, 2),
             "roofline_us": round(t_roof * 1e6, 3), "frac_of_roofline": round(t_roof / per_step_s, 4)}
 
@@ -326,7 +326,7 @@ def run_gpu(args):
     per_launch = measure_problem(torch, prob, 256, 40)
     achieved = prob.bytes / per_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
-    kernel_name = "tc_gemm_kernel<32>" if args.workload == "batch32" else "gemv_mma_kernel<1>"
+    kernel_name = "tc_gemm_kernel<32>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
     traffic = traffic_from_profiles("tc_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
 
     extras = {}
