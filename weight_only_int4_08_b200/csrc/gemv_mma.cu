@@ -399,15 +399,18 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             if constexpr (FAST) {
                 if (rs >= g_next) advance_group();
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int q = 0; q < kRows / 32; ++q) {
+                    // rows 32q + lane of all four chunks; ((32q + lane) >> 1) & 3 == (lane >> 1) & 3
+                    uint32_t R[4][4];
 #pragma unroll
-                    for (int q = 0; q < kRows / 32; ++q) {
-                        // rows 32q + lane; ((32q + lane) >> 1) & 3 == (lane >> 1) & 3
-                        uint32_t R[4];
-                        ptx::ldmatrix_x4_trans(wst + 32 * q * 64 + w_row + 16 * (c ^ w_sw), R);
-                        mma_chunk(c, R[0], R[1], bf[2 * q][0], bf[2 * q][1]);
-                        mma_chunk(c, R[2], R[3], bf[2 * q + 1][0], bf[2 * q + 1][1]);
-                    }
+                    for (int c = 0; c < 4; ++c) ptx::ldmatrix_x4_trans(wst + 32 * q * 64 + w_row + 16 * (c ^ w_sw), R[c]);
+                    // chunks innermost: consecutive MMAs update different accumulators
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            mma_chunk(c, R[c][2 * hh], R[c][2 * hh + 1], bf[2 * q + hh][0], bf[2 * q + hh][1]);
+                }
             } else {
 #pragma unroll
                 for (int h = 0; h < kSteps; ++h) {
@@ -425,10 +428,9 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             }
             // Every lane has read the stage: it can be refilled.
             __syncwarp();
-            if (lane == 0 && !p.stall_loads) {
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                arm_next();
-            }
+            // (The ldmatrix results were consumed above, so the reads are complete before the copy
+            // that overwrites the stage is issued.)
+            if (lane == 0 && !p.stall_loads) arm_next();
         }
         if (g_cur >= g_first && !failed) group_end();
 

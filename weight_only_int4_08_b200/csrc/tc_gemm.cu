@@ -76,6 +76,7 @@ struct TcArgs {
     int* status;           // workspace status word
     int64_t N, K;
     int G, zp_bias, split, mblk, m0;
+    uint32_t magic;        // 0x64006400, passed at run time so that (x & mask) | magic is one logic op
     int stall_loads;       // tests only: the producer issues nothing (every wait runs out)
     uint64_t wait_ns;      // limit on each device-side wait
 };
@@ -102,12 +103,10 @@ __device__ __forceinline__ uint32_t idesc_f16() {
     return (1u << 4) | ((uint32_t)(MN >> 3) << 17) | ((uint32_t)(kBlockN >> 4) << 24);
 }
 
-// Segments of 16-k MMA steps: a segment ends at a group end or at the slab end.
+// The slab's rows; a segment of 16-k MMA steps ends at a group end or at the slab end.
 struct SegIter {
     int64_t k_lo, k_hi;  // slab rows
     int G;
-    __device__ bool starts(int64_t k) const { return k == k_lo || k % G == 0; }
-    __device__ bool ends(int64_t k) const { return k + 16 == k_hi || (k + 16) % G == 0; }
 };
 
 template <int MN>
@@ -190,10 +189,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const int64_t nw = p.N / 8;
         const int64_t word = (int64_t)tile * kTileWords + 4 * warp + (t1 >> 1);  // holds my 4 columns
         const int nib0 = 4 * (t1 & 1);                                           // their first nibble
-        int64_t g_cur = -1;
         const int64_t ngroups = p.K / p.G;
+        // Groups advance one at a time over the slab: g_cur is the open group, g_next_k its end.
+        int64_t g_cur = st_lo * kStageK / p.G - 1, g_next_k = (g_cur + 1) * p.G;
         uint32_t zw_next = 0u;
+        bool have_next = false;
         uint32_t bias0 = 0, bias1 = 0, bias2 = 0, bias3 = 0;
+        const uint32_t magic = p.magic;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
         for (int i = 0; i < nst; ++i) {
             const int s = i % SS, ts = i % kTmemStages;
@@ -214,15 +216,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 #pragma unroll
                 for (int mi = 0; mi < 4; ++mi) {
                     const int64_t kk = (st_lo + i) * kStageK + 32 * h + 8 * mi;   // first k of this matrix
-                    const int64_t g = kk / p.G;
-                    if (g != g_cur) {
+                    if (kk >= g_next_k) {   // G is a multiple of 16, so a group starts here or not at all
+                        const int64_t g = ++g_cur;
+                        g_next_k += p.G;
                         // zero word of this group (prefetched one group ahead), then prefetch the next
                         uint32_t zraw = 0u;
                         if (p.z) {
-                            zraw = (g == g_cur + 1 && g_cur >= 0) ? zw_next : __ldg(p.z + g * nw + word);
-                            if (g + 1 < ngroups) zw_next = __ldg(p.z + (g + 1) * nw + word);
+                            zraw = have_next ? zw_next : __ldg(p.z + g * nw + word);
+                            have_next = g + 1 < ngroups;
+                            if (have_next) zw_next = __ldg(p.z + (g + 1) * nw + word);
                         }
-                        g_cur = g;
                         const uint32_t zw = p.z ? (zraw >> (4 * nib0)) : (uint32_t)p.zp_bias * 0x1111u;
                         // (1024 + z) for low-nibble columns, (1024 + 16 z) for high ones, in both halves
                         bias0 = (0x6400u + (zw & 0xFu)) * 0x00010001u;
@@ -232,10 +235,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     }
                     const uint32_t x = R[mi], y = x >> 8;
                     const uint32_t col = (uint32_t)(ts * 32 + 16 * h + 4 * mi);
-                    ptx::tmem_st_16x128b(lane_base + col, hsub2((x & 0x000F000Fu) | 0x64006400u, bias0),
-                                         hsub2((x & 0x00F000F0u) | 0x64006400u, bias1));
-                    ptx::tmem_st_16x128b(lane_base + (16u << 16) + col, hsub2((y & 0x000F000Fu) | 0x64006400u, bias2),
-                                         hsub2((y & 0x00F000F0u) | 0x64006400u, bias3));
+                    ptx::tmem_st_16x128b(lane_base + col, hsub2((x & 0x000F000Fu) | magic, bias0),
+                                         hsub2((x & 0x00F000F0u) | magic, bias1));
+                    ptx::tmem_st_16x128b(lane_base + (16u << 16) + col, hsub2((y & 0x000F000Fu) | magic, bias2),
+                                         hsub2((y & 0x00F000F0u) | magic, bias3));
                 }
             }
             ptx::tmem_wait_st();
@@ -248,6 +251,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             const uint32_t idesc = idesc_f16<MN>();
             int sg = 0;              // segment counter
             uint32_t acc = 0;
+            // Segments of 16-k steps end at a group boundary or at the slab end; tracked incrementally.
+            int64_t seg_next = (seg.k_lo / p.G + 1) * p.G;   // next group boundary after the slab start
+            bool starts = true;
             for (int i = 0; i < nst; ++i) {
                 const int s = i % SS, ts = i % kTmemStages;
                 if (!ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort, p.wait_ns)) break;
@@ -258,7 +264,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 for (int j = 0; j < 4; ++j) {
                     const int64_t k = (st_lo + i) * kStageK + 16 * j;
                     const int db = sg & 1;
-                    if (seg.starts(k)) {
+                    const bool ends = k + 16 == seg.k_hi || k + 16 == seg_next;
+                    if (k + 16 == seg_next) seg_next += p.G;
+                    if (starts) {
                         if (!ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1, &s_abort, p.wait_ns)) {
                             ok = false;
                             break;
@@ -269,7 +277,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     ptx::mma_f16_ts(tmem + (uint32_t)(C::kDCol + db * MN), tmem + (uint32_t)(ts * 32 + 8 * j),
                                     kmajor_sw128_desc(bbase + 32 * j), idesc, acc);
                     acc = 1;
-                    if (seg.ends(k)) {
+                    starts = ends;
+                    if (ends) {
                         ptx::mma_commit(ptx::smem_addr(&bar_dfull[db]));
                         ++sg;
                     }
@@ -295,18 +304,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         for (int m = 0; m < MN; ++m) tot[m] = 0.f;
         int sg = 0;
         bool ok = true;
-        // Segment ends in order; each segment's scale is loaded one segment ahead.
-        auto seg_end_from = [&](int64_t k) -> int64_t {  // last 16-step of the segment holding k
-            return min(seg.k_hi, (k / p.G + 1) * (int64_t)p.G) - 16;
-        };
-        auto scale_of = [&](int64_t kend) -> float {
-            return fscale * __half2float(p.s[(kend / p.G) * p.N + n]);
-        };
-        int64_t k_end = seg_end_from(seg.k_lo);
-        float sc = scale_of(k_end);
+        // Segment ends in order (group boundaries, tracked incrementally); each segment's scale is
+        // loaded one segment ahead.
+        int64_t g_idx = seg.k_lo / p.G;                    // group of the current segment
+        int64_t bound = (g_idx + 1) * p.G;                 // its end row (or the slab end)
+        auto scale_of = [&](int64_t g) -> float { return fscale * __half2float(p.s[g * p.N + n]); };
+        int64_t k_end = min(seg.k_hi, bound) - 16;
+        float sc = scale_of(g_idx);
         while (k_end >= seg.k_lo && ok) {
-            const int64_t k_next = k_end + 16 < seg.k_hi ? seg_end_from(k_end + 16) : -1;
-            const float sc_next = k_next >= 0 ? scale_of(k_next) : 0.f;
+            const int64_t k_next = k_end + 16 < seg.k_hi ? min(seg.k_hi, bound + p.G) - 16 : -1;
+            const float sc_next = k_next >= 0 ? scale_of(g_idx + 1) : 0.f;
             const int db = sg & 1;
             const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_dfull[db]), (sg >> 1) & 1, &s_abort, p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) {  // warp-uniform: tcgen05.ld is .sync.aligned
@@ -328,6 +335,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             ++sg;
             k_end = k_next;
             sc = sc_next;
+            ++g_idx;
+            bound += p.G;
         }
         // One decision for all 128 epilogue threads (a timeout seen by any of them,
         // or by another role, skips the output), so the named barriers below match.
@@ -494,6 +503,7 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
         args.K = K;
         args.G = G;
         args.zp_bias = zp_bias;
+        args.magic = 0x64006400u;
         args.split = pl.split_k;
         args.mblk = (int)std::min<int64_t>(128, M - m0);
         args.m0 = (int)m0;
