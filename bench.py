@@ -9,9 +9,13 @@ algorithmic bytes (packed weights + scales + zeros + activations + output).
 
 Timing: inputs are resident in HBM; each step reads a different copy of the
 weights, R copies rotating with R * bytes > 2x L2, so every step streams its
-weights from HBM (no L2 flush needed). Steps run back to back from a CUDA graph;
-CUDA events on the launching stream bracket exactly K steps, with a barrier and
-a device synchronize on both sides; the max over ranks is taken.
+weights from HBM (no L2 flush needed). Steps run back to back from a CUDA graph,
+as the layers of a decode step would, with programmatic dependent launch: a step
+may start streaming its weights while the previous one finishes, and reads its
+activations only after it (--no-pdl turns this off; the line also reports the
+per-step time without it). CUDA events on the launching stream bracket exactly
+K steps, with a barrier and a device synchronize on both sides; the max over
+ranks is taken.
 
 Multi-GPU: the layer is run as independent replicas, one per GPU (weak scaling);
 there is no collective on the data path.
@@ -159,11 +163,13 @@ class Problem:
         self.bytes = alg_bytes(self.M, self.K, self.N, self.G, self.asym)
         self.flops = alg_flops(self.M, self.K, self.N)
 
+    pdl = True  # back-to-back steps read weights no step writes: programmatic dependent launch is valid
+
     def step(self, stream=None):
         j = self.i % len(self.bs)
         self.i += 1
         self.w.w4a16_gemm(self.a, self.bs[j], self.ss[j], self.zs[j], self.G, self.zp, out=self.out,
-                          workspace=self.ws, stream=stream)
+                          workspace=self.ws, stream=stream, pdl=self.pdl)
 
     def launches_per_step(self):
         # GEMV for M <= 8; tensor-core GEMM (one launch per 128 rows) above.
@@ -237,6 +243,7 @@ def run_gpu(args):
 
     import weight_only_int4_08_b200 as w
     peaks, peak_src = load_peaks()
+    Problem.pdl = args.pdl
 
     if args.workload == "batch32":
         # batch-32 asymmetric GEMM (tensor cores), weights repacked from the checkpoint layout
@@ -324,6 +331,10 @@ def run_gpu(args):
 
     # kernel duration for the roofline: graph of back-to-back launches, CUDA events
     per_launch = measure_problem(torch, prob, 256, 40)
+    # the same without programmatic dependent launch (each call waits for the previous to end)
+    Problem.pdl = False
+    per_launch_plain = measure_problem(torch, prob, 256, 40)
+    Problem.pdl = args.pdl
     achieved = prob.bytes / per_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
     kernel_name = "tc_gemm_kernel<32>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
@@ -356,6 +367,8 @@ def run_gpu(args):
                    "l2": f"inputs larger than L2: {len(prob.bs)} rotating weight copies "
                          f"({len(prob.bs) * prob.bytes / 1e6:.0f} MB)",
                    "timing": "CUDA graph of back-to-back steps, CUDA events on the launching stream"},
+        "no_pdl": {"us_per_step": round(per_launch_plain * 1e6, 3),
+                   "GB/s": round(prob.bytes / per_launch_plain / 1e9, 1)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else peak_src,
@@ -423,7 +436,7 @@ def run_stack(torch, w, peaks):
         def one_pass():
             for row in layers:
                 for idx, (b, s, k, n) in enumerate(row):
-                    w.w4a16_gemm(acts[0][idx], b, s, None, 128, 8, out=outs[idx], workspace=wss[idx])
+                    w.w4a16_gemm(acts[0][idx], b, s, None, 128, 8, out=outs[idx], workspace=wss[idx], pdl=True)
 
         g = capture(torch, one_pass, 1)
         time_graph(torch, g, 2)
@@ -491,6 +504,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-pdl", dest="pdl", action="store_false",
+                    help="launch every step only after the previous one has finished")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--workload", default="decode_m1", choices=["decode_m1", "batch32"],

@@ -141,14 +141,25 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  *     timeout path only.
  *   wait_limit_us: 0 = the default limit (2 s) on every device-side wait,
  *     else that many microseconds.
+ *   launch_flags: 0 or W4A16_LAUNCH_PDL. With W4A16_LAUNCH_PDL the mma.sync
+ *     GEMV is launched with programmatic dependent launch: it may start while
+ *     the kernel before it on the stream is still running, and streams its
+ *     packed weights, scales and zeros right away; it waits for that kernel to
+ *     finish (and its writes to be visible) before it reads A or writes out
+ *     or the workspace. The caller guarantees that the preceding kernel does
+ *     not write b_packed, scales or qzeros (a GEMM after another GEMM or an
+ *     activation kernel qualifies; a GEMM right after the w4a16_repack that
+ *     produced its weights does not). Other kernels ignore the flag.
  */
 enum { W4A16_KERNEL_AUTO = 0, W4A16_KERNEL_GEMV = 1, W4A16_KERNEL_TC = 2, W4A16_KERNEL_GEMV_FMA = 3 };
 enum { W4A16_DEBUG_STALL_LOADS = 1 };
+enum { W4A16_LAUNCH_PDL = 1 };
 typedef struct {
     int32_t kernel;
     int32_t split_k;
     uint32_t debug_flags;
     uint32_t wait_limit_us;
+    uint32_t launch_flags;
 } w4a16_gemm_options;
 
 /* Workspace bytes for w4a16_gemm_ex with these options (NULL opts = automatic). */

@@ -27,10 +27,11 @@ KERNEL_AUTO, KERNEL_GEMV, KERNEL_TC, KERNEL_GEMV_FMA = 0, 1, 2, 3
 
 class W4A16Options(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("split_k", ctypes.c_int32), ("debug_flags", ctypes.c_uint32),
-                ("wait_limit_us", ctypes.c_uint32)]
+                ("wait_limit_us", ctypes.c_uint32), ("launch_flags", ctypes.c_uint32)]
 
 
 DEBUG_STALL_LOADS = 1
+LAUNCH_PDL = 1
 
 
 _p, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
@@ -89,11 +90,11 @@ def _dev(t, name, dtype):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _opts(kernel, split_k, debug_flags=0, wait_limit_us=0):
-    if kernel is None and not split_k and not debug_flags and not wait_limit_us:
+def _opts(kernel, split_k, debug_flags=0, wait_limit_us=0, launch_flags=0):
+    if kernel is None and not split_k and not debug_flags and not wait_limit_us and not launch_flags:
         return None
     return ctypes.byref(W4A16Options(int(kernel or KERNEL_AUTO), int(split_k or 0), int(debug_flags),
-                                     int(wait_limit_us)))
+                                     int(wait_limit_us), int(launch_flags)))
 
 
 def w4a16_status_string(status: int) -> str:
@@ -130,8 +131,11 @@ def w4a16_repack(ckpt_nk8: torch.Tensor, N: int, K: int, out: torch.Tensor | Non
 def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qzeros: torch.Tensor | None,
                group_size: int, zp_bias: int = 8, out: torch.Tensor | None = None,
                workspace: torch.Tensor | None = None, stream=None, kernel=None, split_k: int = 0,
-               debug_flags: int = 0, wait_limit_us: int = 0):
-    """out[M, N] = fp16(fp32(a) @ ((q - z) * s)) on the GPU (see include/w4a16.h)."""
+               debug_flags: int = 0, wait_limit_us: int = 0, pdl: bool = False):
+    """out[M, N] = fp16(fp32(a) @ ((q - z) * s)) on the GPU (see include/w4a16.h).
+
+    pdl=True sets W4A16_LAUNCH_PDL: only when the kernel before this call on the stream does not
+    write b_packed, scales or qzeros."""
     pa = _dev(a, "a", (torch.float16,))
     pb = _dev(b_packed, "b_packed", (torch.int32, torch.uint32))
     ps = _dev(scales, "scales", (torch.float16,))
@@ -154,7 +158,7 @@ def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qz
     if workspace is None:
         workspace = alloc_workspace(M, N, K, group_size, a.device, kernel, split_k)
     pw = _dev(workspace, "workspace", (torch.uint8,))
-    o = _opts(kernel, split_k, debug_flags, wait_limit_us)
+    o = _opts(kernel, split_k, debug_flags, wait_limit_us, LAUNCH_PDL if pdl else 0)
     args = (pa, pb, ps, pz, M, N, K, group_size, zp_bias, po, pw, workspace.numel(), _stream_ptr(stream))
     rc = lib.w4a16_gemm(*args) if o is None else lib.w4a16_gemm_ex(*args, o)
     _check(rc, "w4a16_gemm")

@@ -22,6 +22,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 struct WaitPolicy {
     uint64_t limit_ns;
     int stall_loads;
+    int pdl;  // launch with programmatic dependent launch (W4A16_LAUNCH_PDL)
 };
 
 struct GemvPlan {

@@ -17,18 +17,19 @@
 // multiply-adds. The MMA's batch dimension (8) is padded for M < 8.
 //
 // Work decomposition (stream-K): the weight matrix is cut into units of one
-// 128-column tile x 64 rows (4 KB of packed weights), ordered tile by tile
+// 128-column tile x 128 rows (8 KB of packed weights), ordered tile by tile
 // along K. A single wave of resident CTAs takes equal contiguous runs of that
 // order, so every SM streams the same number of bytes whatever N and K are. A
 // CTA's run covers pieces ("fragments") of one to a few tiles; within a
 // fragment its 8 warps take equal runs of units, each through a private ring
 // of two shared-memory stages filled by 2-D TMA loads (weights with 64-byte
 // swizzle, which makes the transposed ldmatrix reads bank-conflict free, and
-// the activations of the same 64 rows) and tracked by one mbarrier per stage.
-// The stage shape follows a measurement on B200: streaming a 29 MB matrix,
-// TMA boxes of 64 B x 16..32 rows ran up to 2x slower than 4 KB boxes, and
-// about 128 KB in flight per SM was enough; more small boxes in flight made it
-// slower. Scales and zero words are copied one group ahead into a small
+// the activations of the same rows) and tracked by one mbarrier per stage.
+// The stage shape follows measurements on B200: streaming a 29 MB matrix,
+// TMA boxes of 64 B x 16..32 rows ran up to 2x slower than boxes of 4 KB and
+// more, and about 128 KB in flight per SM was enough; and one resident CTA per
+// SM with 128-row stages needs fewer instructions per byte (no register cap,
+// half the per-stage bookkeeping) than two CTAs with 64-row stages. Scales and zero words are copied one group ahead into a small
 // per-warp shared buffer (cp.async); each group's scaled sums are added to
 // fp32 totals kept in shared memory. At the end of a fragment the warps are
 // reduced in warp order; a tile covered by one CTA is
@@ -50,19 +51,22 @@
 namespace w4a16 {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = 8;
+#ifndef W4A16_SK_WARPS
+#define W4A16_SK_WARPS 8
+#endif
+constexpr int kWarps = W4A16_SK_WARPS;
+constexpr int kThreads = 32 * kWarps;
 constexpr int kTileN = 128;
 constexpr int kTileWords = kTileN / 8;            // 16 packed words = 64 B per row
 #ifndef W4A16_SK_ROWS
-#define W4A16_SK_ROWS 64
+#define W4A16_SK_ROWS 128
 #endif
 #ifndef W4A16_SK_RING
 #define W4A16_SK_RING 2
 #endif
 constexpr int kRows = W4A16_SK_ROWS;              // rows per unit / TMA stage (a multiple of 32)
 constexpr int kSteps = kRows / 16;                // 16-row MMA steps per stage
-constexpr int kWStage = kRows * kTileWords * 4;   // packed weight bytes per stage (4 KB)
+constexpr int kWStage = kRows * kTileWords * 4;   // packed weight bytes per stage (8 KB)
 constexpr int kRing = W4A16_SK_RING;              // stages in flight per warp
 constexpr int kWRingBytes = kWarps * kRing * kWStage;
 constexpr int kMaxCluster = 8;                    // portable thread-block cluster size
@@ -71,7 +75,7 @@ constexpr int kMaxCluster = 8;                    // portable thread-block clust
 // the rows are loaded with 128-byte swizzle (so that ldmatrix reads of 8 rows hit 8 different
 // bank groups), which needs 1024-byte aligned slots; up to four rows the conflicts are cheaper
 // than the padding.
-__host__ __device__ constexpr bool a_swizzled(int mt) { return mt > 4; }
+__host__ __device__ constexpr bool a_swizzled(int mt) { return mt > 4 && kRows == 64; }
 __host__ __device__ constexpr int a_slot_bytes(int mt) { return a_swizzled(mt) ? 1024 : 2 * kRows * mt; }
 // Per warp, two group buffers: the tile's 128 scales (256 B) and 16 zero words (64 B).
 constexpr int kGrpBytes = 2 * kTileN + 4 * kTileWords;
@@ -176,10 +180,10 @@ __device__ __forceinline__ float ld_cluster(uint32_t addr) {
 }
 
 #ifndef W4A16_SK_MIN_CTAS
-#define W4A16_SK_MIN_CTAS 2
+#define W4A16_SK_MIN_CTAS 1   // one resident CTA per SM: no register cap (a cap of 128 cost ~15 % in moves)
 #endif
-// FAST: the group size is a multiple of the 64-row unit, so a group starts only at a unit start
-// (and K is a multiple of 64); otherwise groups are tracked per 16-row step.
+// FAST: the group size is a multiple of the unit (kRows), so a group starts only at a unit start
+// (and K is a multiple of kRows); otherwise groups are tracked per 16-row step.
 template <int MT, bool FAST>
 __global__ void __launch_bounds__(kThreads, W4A16_SK_MIN_CTAS)
 gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap amap, SkArgs p) {
@@ -201,7 +205,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     unsigned char* grp = grps + warp * 2 * kGrpBytes;
     const int nblk = p.nblk, G = p.G, K = (int)p.K;
     const int nw = (int)(p.N / 8);
-    // My cluster owns tiles [tile_lo, tile_hi); its units (tile-major, 64-row blocks) are split in
+    // My cluster owns tiles [tile_lo, tile_hi); its units (tile-major, kRows-row blocks) are split in
     // S equal contiguous runs, mine being run `rank`. Unit counts fit in 32 bits (the weights would
     // not fit in memory otherwise; the host checks).
     const int S = (int)cluster_nctarank(), rank = (int)cluster_ctarank();
@@ -234,12 +238,17 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     const uint32_t w0 = ptx::smem_addr(wring + warp * kRing * kWStage);
     const uint32_t a0 = ptx::smem_addr(aring + warp * kRing * kASlot);
 
-    // Load issue (lane 0): a cursor over this warp's units, one stage per unit.
+    // With programmatic dependent launch the next kernel on the stream may start now; it waits for
+    // this one to finish before it touches anything this one writes.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // Load issue (lane 0): a cursor over this warp's units, one stage per unit. A stage's barrier
+    // expects the weight box and the activation box; the activations may be issued later.
     int pf = 0, pkb = 0, phi = 0, armed = 0;
     frag_lo_hi(0, pkb, phi);
-    auto arm_next = [&]() {
+    auto arm_w = [&]() -> int {   // the unit's k-block, or -1 when the warp has no more units
         while (pkb >= phi) {
-            if (pf + 1 >= nfrag) return;
+            if (pf + 1 >= nfrag) return -1;
             ++pf;
             frag_lo_hi(pf, pkb, phi);
         }
@@ -247,14 +256,31 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         const uint32_t bar = bar0 + 8 * slot;
         ptx::mbar_arrive_expect_tx(bar, (uint32_t)(kWStage + 2 * kRows * MT));
         ptx::tma_load_2d(w0 + slot * kWStage, &bmap, (t0 + pf) * kTileWords, pkb * kRows, bar);
-        ptx::tma_load_2d(a0 + slot * kASlot, &amap, pkb * kRows, 0, bar);
-        ++pkb;
         ++armed;
+        return pkb++;
     };
+    auto issue_a = [&](int slot, int kb) {
+        ptx::tma_load_2d(a0 + slot * kASlot, &amap, kb * kRows, 0, bar0 + 8 * slot);
+    };
+    auto arm_next = [&]() {
+        const int slot = armed % kRing;
+        const int kb = arm_w();
+        if (kb >= 0) issue_a(slot, kb);
+    };
+    // Prologue: the first stages' weights (independent of any earlier kernel) go out first; the
+    // activations, written by the kernel before this one, only after it has completed.
+    int first_kb[kRing];
     if (lane == 0 && !p.stall_loads) {
         ptx::prefetch_tensormap(&bmap);
         ptx::prefetch_tensormap(&amap);
-        for (int j = 0; j < kRing; ++j) arm_next();
+#pragma unroll
+        for (int j = 0; j < kRing; ++j) first_kb[j] = arm_w();
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (lane == 0 && !p.stall_loads) {
+#pragma unroll
+        for (int j = 0; j < kRing; ++j)
+            if (first_kb[j] >= 0) issue_a(j, first_kb[j]);
     }
 
     const int zshift = 16 * (g & 1);  // my first column is nibble 4 (g & 1) of its zero word
@@ -278,8 +304,9 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // zero row past MT; the second ldmatrix of a stage reads 4 blocks further.
     const int br = lane & 7, bc = lane >> 3;
     const uint32_t b_off = br < MT ? a0 + br * 2 * kRows : ptx::smem_addr(&s_zero);
-    const uint32_t b_col0 = br < MT ? 16 * (a_swizzled(MT) ? (bc ^ br) : bc) : 0;
-    const uint32_t b_col1 = br < MT ? 16 * (a_swizzled(MT) ? ((4 + bc) ^ br) : (4 + bc)) : 0;
+    auto b_col = [&](int h2) -> uint32_t {   // 16-byte column block 4 h2 + bc of row br
+        return br < MT ? 16 * (a_swizzled(MT) ? ((4 * h2 + bc) ^ br) : (4 * h2 + bc)) : 0;
+    };
     const uint32_t b_slot = br < MT ? kASlot : 0;
     // Weight ldmatrix.trans address of lane (row lane, 16-byte chunk c) under the 64-byte swizzle:
     // row r holds chunk c at chunk c ^ ((r >> 1) & 3).
@@ -383,18 +410,14 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             const uint32_t wst = w0 + slot * kWStage;
             // B fragments (batch row g, k-pairs t and t + 4 of each 16-row step), two steps per ldmatrix.
             uint32_t bf[kSteps][2];
-            {
+#pragma unroll
+            for (int h2 = 0; h2 < kSteps / 2; ++h2) {
                 uint32_t B[4];
-                ldmatrix_x4(b_off + slot * b_slot + b_col0, B);
-                bf[0][0] = B[0];
-                bf[0][1] = B[1];
-                bf[1][0] = B[2];
-                bf[1][1] = B[3];
-                ldmatrix_x4(b_off + slot * b_slot + b_col1, B);
-                bf[2][0] = B[0];
-                bf[2][1] = B[1];
-                bf[3][0] = B[2];
-                bf[3][1] = B[3];
+                ldmatrix_x4(b_off + slot * b_slot + b_col(h2), B);
+                bf[2 * h2][0] = B[0];
+                bf[2 * h2][1] = B[1];
+                bf[2 * h2 + 1][0] = B[2];
+                bf[2 * h2 + 1][1] = B[3];
             }
             if constexpr (FAST) {
                 if (rs >= g_next) advance_group();
@@ -665,13 +688,15 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         cfg.blockDim = dim3(kThreads);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = (unsigned)pl.cluster;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = wp.pdl ? 2 : 1;
         e = cudaLaunchKernelEx(&cfg, k, bmap, amap, args);
         if (e != cudaSuccess) return e;
     }

@@ -219,6 +219,7 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
         return fail_arg("unknown kernel option");
     if (opts && (opts->split_k < 0 || opts->split_k > 256)) return fail_arg("split_k must be in 0..256");
     if (opts && (opts->debug_flags & ~(uint32_t)W4A16_DEBUG_STALL_LOADS)) return fail_arg("unknown debug flag");
+    if (opts && (opts->launch_flags & ~(uint32_t)W4A16_LAUNCH_PDL)) return fail_arg("unknown launch flag");
     if (!aligned(a, 2) || !aligned(scales, 2) || !aligned(out, 2)) return fail_arg("fp16 pointers must be 2-byte aligned");
     if (!aligned(b_packed, 4) || (qzeros && !aligned(qzeros, 4))) return fail_arg("int32 pointers must be 4-byte aligned");
     const size_t a_bytes = (size_t)M * K * 2, b_bytes = (size_t)K * N / 2, s_bytes = (size_t)(K / group_size) * N * 2;
@@ -256,6 +257,7 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
     WaitPolicy wp;
     wp.limit_ns = (opts && opts->wait_limit_us) ? (uint64_t)opts->wait_limit_us * 1000ull : 2000000000ull;
     wp.stall_loads = (opts && (opts->debug_flags & W4A16_DEBUG_STALL_LOADS)) ? 1 : 0;
+    wp.pdl = (opts && (opts->launch_flags & W4A16_LAUNCH_PDL)) ? 1 : 0;
     if (c.kernel == W4A16_KERNEL_TC) {
         e = launch_tc(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
                       static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K, group_size,
