@@ -176,6 +176,14 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t saddr, uint32_t (&r)[
                  : "memory");
 }
 
+// ---- warp leader -------------------------------------------------------------------
+// True in exactly one lane of the (converged) warp.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}" : "=r"(pred));
+    return pred != 0;
+}
+
 // ---- named barrier among a subset of warps ---------------------------------------
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

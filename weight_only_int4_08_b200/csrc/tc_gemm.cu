@@ -162,26 +162,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
+        // Converged loop, one elected lane issuing (as for the MMA warp).
+        const bool leader = ptx::elect_one();
+        if (leader) {
             ptx::prefetch_tensormap(&amap);
             ptx::prefetch_tensormap(&wmap);
-            const uint32_t tx = kWStageBytes + C::kBStageBytes;
-            int issued = 0;
-            for (int i = 0; i < nst && !p.stall_loads; ++i) {
-                const int s = i % SS;
-                if (!ptx::mbar_wait(ptx::smem_addr(&bar_empty[s]), ((i / SS) & 1) ^ 1, &s_abort, p.wait_ns)) break;
+        }
+        const uint32_t tx = kWStageBytes + C::kBStageBytes;
+        int issued = 0;
+        for (int i = 0; i < nst && !p.stall_loads; ++i) {
+            const int s = i % SS;
+            const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_empty[s]), ((i / SS) & 1) ^ 1, &s_abort, p.wait_ns);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            if (leader) {
                 const uint32_t full = ptx::smem_addr(&bar_full[s]);
                 ptx::mbar_arrive_expect_tx(full, tx);
                 const int32_t k0 = (int32_t)((st_lo + i) * kStageK);
                 ptx::tma_load_2d(ptx::smem_addr(s_w + (size_t)s * kWStageBytes), &wmap, tile * kTileWords, k0, full);
                 ptx::tma_load_2d(ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes), &amap, k0, p.m0, full);
-                issued = i + 1;
             }
-            if (s_abort) {  // let copies already issued land before the CTA leaves
-                volatile int dummy = 0;
-                for (int i = max(0, issued - SS); i < issued; ++i)
-                    ptx::mbar_wait(ptx::smem_addr(&bar_full[i % SS]), (i / SS) & 1, &dummy, p.wait_ns);
-            }
+            __syncwarp();
+            issued = i + 1;
+        }
+        if (s_abort && leader) {  // let copies already issued land before the CTA leaves
+            volatile int dummy = 0;
+            for (int i = max(0, issued - SS); i < issued; ++i)
+                ptx::mbar_wait(ptx::smem_addr(&bar_full[i % SS]), (i / SS) & 1, &dummy, p.wait_ns);
         }
     } else if (warp < 4) {
         // -------------------------------------------------------- dequantisers
@@ -247,51 +253,62 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         }
     } else if (warp == 5) {
         // ----------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_f16<MN>();
-            int sg = 0;              // segment counter
-            uint32_t acc = 0;
-            // Segments of 16-k steps end at a group boundary or at the slab end; tracked incrementally.
-            int64_t seg_next = (seg.k_lo / p.G + 1) * p.G;   // next group boundary after the slab start
-            bool starts = true;
-            for (int i = 0; i < nst; ++i) {
-                const int s = i % SS, ts = i % kTmemStages;
-                if (!ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort, p.wait_ns)) break;
-                if (!ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns)) break;
-                ptx::tc_fence_after();
-                const uint32_t bbase = ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes);
-                bool ok = true;
-                for (int j = 0; j < 4; ++j) {
-                    const int64_t k = (st_lo + i) * kStageK + 16 * j;
-                    const int db = sg & 1;
-                    const bool ends = k + 16 == seg.k_hi || k + 16 == seg_next;
-                    if (k + 16 == seg_next) seg_next += p.G;
-                    if (starts) {
-                        if (!ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1, &s_abort, p.wait_ns)) {
-                            ok = false;
-                            break;
-                        }
-                        ptx::tc_fence_after();
-                        acc = 0;
+        // The whole warp runs the loop (so the operands stay warp-uniform) and one elected lane
+        // issues the MMAs and commits: measured on B200, issuing from a lane-0-only branch cost
+        // about 240 cycles per tcgen05.mma.
+        const bool leader = ptx::elect_one();
+        const uint32_t idesc = idesc_f16<MN>();
+        int sg = 0;              // segment counter
+        uint32_t acc = 0;
+        // Segments of 16-k steps end at a group boundary or at the slab end; tracked incrementally.
+        int64_t seg_next = (seg.k_lo / p.G + 1) * p.G;   // next group boundary after the slab start
+        bool starts = true;
+        for (int i = 0; i < nst; ++i) {
+            const int s = i % SS, ts = i % kTmemStages;
+            bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort, p.wait_ns);
+            okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            ptx::tc_fence_after();
+            const uint32_t bbase = ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes);
+            bool ok = true;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t k = (st_lo + i) * kStageK + 16 * j;
+                const int db = sg & 1;
+                const bool ends = k + 16 == seg.k_hi || k + 16 == seg_next;
+                if (k + 16 == seg_next) seg_next += p.G;
+                if (starts) {
+                    const bool okd = ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1, &s_abort,
+                                                    p.wait_ns);
+                    if (!__all_sync(0xffffffffu, okd)) {
+                        ok = false;
+                        break;
                     }
+                    ptx::tc_fence_after();
+                    acc = 0;
+                }
+                if (leader)
                     ptx::mma_f16_ts(tmem + (uint32_t)(C::kDCol + db * MN), tmem + (uint32_t)(ts * 32 + 8 * j),
                                     kmajor_sw128_desc(bbase + 32 * j), idesc, acc);
-                    acc = 1;
-                    starts = ends;
-                    if (ends) {
-                        ptx::mma_commit(ptx::smem_addr(&bar_dfull[db]));
-                        ++sg;
-                    }
+                acc = 1;
+                starts = ends;
+                if (ends) {
+                    if (leader) ptx::mma_commit(ptx::smem_addr(&bar_dfull[db]));
+                    ++sg;
                 }
+            }
+            if (leader) {
                 ptx::mma_commit(ptx::smem_addr(&bar_empty[s]));
                 ptx::mma_commit(ptx::smem_addr(&bar_aempty[ts]));
-                if (!ok) break;
             }
-            // Wait for every MMA issued above before TMEM can be released.
-            volatile int dummy = 0;
-            ptx::mma_commit(ptx::smem_addr(&bar_drain));
-            ptx::mbar_wait(ptx::smem_addr(&bar_drain), 0, &dummy, p.wait_ns);
+            __syncwarp();
+            if (!ok) break;
         }
+        // Wait for every MMA issued above before TMEM can be released.
+        if (leader) ptx::mma_commit(ptx::smem_addr(&bar_drain));
+        __syncwarp();
+        volatile int dummy = 0;
+        ptx::mbar_wait(ptx::smem_addr(&bar_drain), 0, &dummy, p.wait_ns);
     } else {
         // -------------------------------------------------------------- epilogue
         const int sub = warp & 3;                           // TMEM lanes 32 sub .. 32 sub + 31
