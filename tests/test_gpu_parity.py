@@ -134,11 +134,29 @@ def test_odd_shapes(w, M, K, N, G, sym):
 
 
 @pytest.mark.parametrize("G", [16, 32, 48, 64, 80, 128, 192, 256])
-@pytest.mark.parametrize("M", [1, 3])
+@pytest.mark.parametrize("M", [1, 3, 12, 16])
 def test_gemv_group_sizes(w, G, M):
     # groups that are and are not multiples of the 64-row load unit; K spans several groups
     c = synth.make_case(M, 8 * G, 384, G, sym=False, seed=G + M)
     assert_close(run(w, c, kernel=w.KERNEL_GEMV), ref(c), f"GEMV G={G} M={M}")
+
+
+@pytest.mark.parametrize("M,K,N,G,sym", [
+    (9, 512, 384, 64, False),      # one 16-row block, two batch tiles (the second partly empty)
+    (13, 640, 544, 80, True),      # groups straddle the 64-row stages; ragged column tile
+    (16, 1024, 256, 16, False),
+    (17, 512, 384, 128, False),    # blocks of 16 and 1 rows (different stage heights)
+    (40, 768, 256, 48, True),      # blocks of 16, 16 and 8 rows
+])
+def test_gemv_two_batch_tiles(w, M, K, N, G, sym):
+    c = synth.make_case(M, K, N, G, sym=sym, seed=M * 31 + K)
+    assert_close(run(w, c, kernel=w.KERNEL_GEMV), ref(c), f"GEMV {M}x{K}x{N} G{G}")
+
+
+@pytest.mark.parametrize("MT", list(range(9, 17)))
+def test_gemv_every_row_count_to_16(w, MT):
+    c = synth.make_case(MT, 1024, 512, 128, sym=(MT % 2 == 0), seed=70 + MT)
+    assert_close(run(w, c), ref(c), f"GEMV M={MT}")
 
 
 @pytest.mark.parametrize("split", [1, 2, 3, 7, 33, 256])

@@ -25,7 +25,7 @@ def w():
     return mod
 
 
-def test_config3_m16_auto_uses_tensor_cores(w):
+def test_config3_m16_auto_and_tensor_cores(w):
     c = synth.config3(16)
     assert_close(run(w, c), ref(c), "config3 M=16")
     assert_close(run(w, c, kernel=w.KERNEL_TC), ref(c), "config3 M=16 forced")

@@ -64,28 +64,34 @@ constexpr int kTileWords = kTileN / 8;            // 16 packed words = 64 B per 
 #ifndef W4A16_SK_RING
 #define W4A16_SK_RING 2
 #endif
-constexpr int kRows = W4A16_SK_ROWS;              // rows per unit / TMA stage (a multiple of 32)
-constexpr int kSteps = kRows / 16;                // 16-row MMA steps per stage
-constexpr int kWStage = kRows * kTileWords * 4;   // packed weight bytes per stage (8 KB)
 constexpr int kRing = W4A16_SK_RING;              // stages in flight per warp
-constexpr int kWRingBytes = kWarps * kRing * kWStage;
 constexpr int kMaxCluster = 8;                    // portable thread-block cluster size
+constexpr int kMaxMT = 16;                        // activation rows per launch: two 8-row MMA tiles
 
-// Activation slot of one stage: MT rows x kRows fp16 (128 B per row). With more than four rows
-// the rows are loaded with 128-byte swizzle (so that ldmatrix reads of 8 rows hit 8 different
-// bank groups), which needs 1024-byte aligned slots; up to four rows the conflicts are cheaper
-// than the padding.
-__host__ __device__ constexpr bool a_swizzled(int mt) { return mt > 4 && kRows == 64; }
-__host__ __device__ constexpr int a_slot_bytes(int mt) { return a_swizzled(mt) ? 1024 : 2 * kRows * mt; }
+// MMA batch tiles (8 activation rows each) of a launch of MT rows.
+__host__ __device__ constexpr int n_tiles(int mt) { return (mt + 7) / 8; }
+// Rows per unit / TMA stage (a multiple of 32): 128 for one batch tile; 64 for two, so that the
+// larger activation stages and totals still fit one CTA's shared memory.
+__host__ __device__ constexpr int rows_for(int mt) { return mt > 8 ? 64 : W4A16_SK_ROWS; }
+__host__ __device__ constexpr int wstage_bytes(int mt) { return rows_for(mt) * kTileWords * 4; }
+// Activation slot of one stage: MT rows x rows_for(MT) fp16. With 64-row stages (128 B per row)
+// and more than four rows the rows are loaded with 128-byte swizzle (so that ldmatrix reads of 8
+// rows hit 8 different bank groups), which needs 1024-byte aligned slots; otherwise the few
+// conflicts are cheaper than the padding.
+__host__ __device__ constexpr bool a_swizzled(int mt) { return mt > 4 && rows_for(mt) == 64; }
+__host__ __device__ constexpr int a_slot_bytes(int mt) {
+    return a_swizzled(mt) ? (2 * 64 * mt + 1023) / 1024 * 1024 : 2 * rows_for(mt) * mt;
+}
 // Per warp, two group buffers: the tile's 128 scales (256 B) and 16 zero words (64 B).
 constexpr int kGrpBytes = 2 * kTileN + 4 * kTileWords;
-// Accumulator values per thread kept across groups: chunk c, entry i of the MMA accumulators
-// (only the even entries, batch 2t, matter for one activation row).
-__host__ __device__ constexpr int tot_per_chunk(int mt) { return mt > 1 ? 8 : 4; }
+// Accumulator values per thread and chunk kept across groups: entry i of each batch tile's MMA
+// accumulators (only the even entries, batch 2t, matter for one activation row).
+__host__ __device__ constexpr int tot_per_tile(int mt) { return mt > 1 ? 8 : 4; }
+__host__ __device__ constexpr int tot_per_chunk(int mt) { return tot_per_tile(mt) * n_tiles(mt); }
 // Dynamic shared memory: weight ring, activation ring, fp32 totals, group buffers, and the
 // warp-reduced sums of the (at most two) fragments shared with other CTAs.
 __host__ __device__ constexpr size_t sk_smem_bytes(int mt) {
-    return (size_t)kWRingBytes + (size_t)kWarps * kRing * a_slot_bytes(mt) +
+    return (size_t)kWarps * kRing * (wstage_bytes(mt) + a_slot_bytes(mt)) +
            (size_t)kWarps * 4 * tot_per_chunk(mt) * 32 * 4 + (size_t)kWarps * 2 * kGrpBytes + 2 * (size_t)mt * kTileN * 4;
 }
 
@@ -187,7 +193,13 @@ __device__ __forceinline__ float ld_cluster(uint32_t addr) {
 template <int MT, bool FAST>
 __global__ void __launch_bounds__(kThreads, W4A16_SK_MIN_CTAS)
 gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap amap, SkArgs p) {
+    constexpr int kRows = rows_for(MT);            // rows per unit / stage
+    constexpr int kSteps = kRows / 16;             // 16-row MMA steps per stage
+    constexpr int kWStage = wstage_bytes(MT);
+    constexpr int kWRingBytes = kWarps * kRing * kWStage;
     constexpr int kASlot = a_slot_bytes(MT);
+    constexpr int NT = n_tiles(MT);                // 8-row batch tiles
+    constexpr int NB = tot_per_tile(MT);
     constexpr int NI = tot_per_chunk(MT);
     extern __shared__ __align__(1024) unsigned char s_dyn[];
     unsigned char* wring = s_dyn;                                        // [warp][kRing][kRows][64 B], 64-byte swizzle
@@ -300,14 +312,16 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
         for (int c = 0; c < 4; ++c) set_bias(c, (uint32_t)p.zp_bias * 0x1111u);
     }
-    // B-fragment ldmatrix address of lane (row lane % 8, 8-k block lane / 8) in ring slot 0, or the
-    // zero row past MT; the second ldmatrix of a stage reads 4 blocks further.
+    // B-fragment ldmatrix address of lane (activation row 8 nt + lane % 8, 8-k block lane / 8) in
+    // ring slot 0, or the zero row past MT; each ldmatrix covers two 16-row steps.
     const int br = lane & 7, bc = lane >> 3;
-    const uint32_t b_off = br < MT ? a0 + br * 2 * kRows : ptx::smem_addr(&s_zero);
-    auto b_col = [&](int h2) -> uint32_t {   // 16-byte column block 4 h2 + bc of row br
-        return br < MT ? 16 * (a_swizzled(MT) ? ((4 * h2 + bc) ^ br) : (4 * h2 + bc)) : 0;
+    auto b_off = [&](int nt) -> uint32_t {
+        return 8 * nt + br < MT ? a0 + (8 * nt + br) * 2 * kRows : ptx::smem_addr(&s_zero);
     };
-    const uint32_t b_slot = br < MT ? kASlot : 0;
+    auto b_col = [&](int nt, int h2) -> uint32_t {   // 16-byte column block 4 h2 + bc of that row
+        return 8 * nt + br < MT ? 16 * (a_swizzled(MT) ? ((4 * h2 + bc) ^ br) : (4 * h2 + bc)) : 0;
+    };
+    auto b_slot = [&](int nt) -> uint32_t { return 8 * nt + br < MT ? kASlot : 0; };
     // Weight ldmatrix.trans address of lane (row lane, 16-byte chunk c) under the 64-byte swizzle:
     // row r holds chunk c at chunk c ^ ((r >> 1) & 3).
     const uint32_t w_row = lane * 64;
@@ -324,7 +338,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         const bool s_ok = (int64_t)tile * kTileN + 32 * (lane / 8) < p.N;
         const bool z_ok = p.z && lane < kTileWords && tile * kTileWords + lane < nw;
 
-        float acc[4][8];
+        float acc[4][NT][8];
 #pragma unroll
         for (int k = 0; k < 4 * NI; ++k) tmine[32 * k] = 0.f;
 
@@ -351,11 +365,13 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
                 const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
                 const float sj[4] = {s01.x, s01.y, s23.x, s23.y};
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if (MT > 1 || (i & 1) == 0) {
-                        float* tp = tmine + 32 * (c * NI + (MT > 1 ? i : i / 2));
-                        *tp = fmaf(sj[i >> 1], acc[c][i], *tp);
-                    }
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if (MT > 1 || (i & 1) == 0) {
+                            float* tp = tmine + 32 * (c * NI + nt * NB + (MT > 1 ? i : i / 2));
+                            *tp = fmaf(sj[i >> 1], acc[c][nt][i], *tp);
+                        }
             }
         };
         // Start group gg (its buffer was filled one group earlier) and prefetch the next one.
@@ -367,7 +383,9 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             for (int c = 0; c < 4; ++c) {
                 if (p.z) set_bias(c, *reinterpret_cast<const uint32_t*>(gb + 2 * kTileN + 4 * (4 * c + g / 2)) >> zshift);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[c][i] = 0.f;
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[c][nt][i] = 0.f;
             }
             if (g_next < rend) load_group(gg + 1);   // g_next is the first row of group gg + 1
         };
@@ -378,14 +396,18 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             group_start(g_cur);
         };
         // Dequantise two 8-row matrices of chunk c (k-rows r..r+7 in x0, r+8..r+15 in x1) and
-        // multiply them with the activation fragment (b0, b1).
-        auto mma_chunk = [&](int c, uint32_t x0, uint32_t x1, uint32_t b0, uint32_t b1) {
+        // multiply them with the activation fragments of 16-row step h (one per batch tile).
+        uint32_t bf[kSteps][NT][2];
+        auto mma_chunk = [&](int c, uint32_t x0, uint32_t x1, int h) {
             {
                 const uint32_t e0a = hsub2((x0 & 0x000F000Fu) | magic, bias[c][0]);
                 const uint32_t e1a = hfma2((x0 & 0x00F000F0u) | magic, kSixteenth, bias[c][1]);
                 const uint32_t e0b = hsub2((x1 & 0x000F000Fu) | magic, bias[c][0]);
                 const uint32_t e1b = hfma2((x1 & 0x00F000F0u) | magic, kSixteenth, bias[c][1]);
-                mma16816(acc[c][0], acc[c][1], acc[c][2], acc[c][3], e0a, e1a, e0b, e1b, b0, b1);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma16816(acc[c][nt][0], acc[c][nt][1], acc[c][nt][2], acc[c][nt][3], e0a, e1a, e0b, e1b,
+                             bf[h][nt][0], bf[h][nt][1]);
             }
             {
                 const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
@@ -393,7 +415,10 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
                 const uint32_t e3a = hfma2((y0 & 0x00F000F0u) | magic, kSixteenth, bias[c][3]);
                 const uint32_t e2b = hsub2((y1 & 0x000F000Fu) | magic, bias[c][2]);
                 const uint32_t e3b = hfma2((y1 & 0x00F000F0u) | magic, kSixteenth, bias[c][3]);
-                mma16816(acc[c][4], acc[c][5], acc[c][6], acc[c][7], e2a, e3a, e2b, e3b, b0, b1);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma16816(acc[c][nt][4], acc[c][nt][5], acc[c][nt][6], acc[c][nt][7], e2a, e3a, e2b, e3b,
+                             bf[h][nt][0], bf[h][nt][1]);
             }
         };
 
@@ -408,17 +433,19 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             ++consumed;
             const int rs = kb * kRows;
             const uint32_t wst = w0 + slot * kWStage;
-            // B fragments (batch row g, k-pairs t and t + 4 of each 16-row step), two steps per ldmatrix.
-            uint32_t bf[kSteps][2];
+            // B fragments (batch row 8 nt + g, k-pairs t and t + 4 of each 16-row step), two steps per
+            // ldmatrix.
 #pragma unroll
-            for (int h2 = 0; h2 < kSteps / 2; ++h2) {
-                uint32_t B[4];
-                ldmatrix_x4(b_off + slot * b_slot + b_col(h2), B);
-                bf[2 * h2][0] = B[0];
-                bf[2 * h2][1] = B[1];
-                bf[2 * h2 + 1][0] = B[2];
-                bf[2 * h2 + 1][1] = B[3];
-            }
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int h2 = 0; h2 < kSteps / 2; ++h2) {
+                    uint32_t B[4];
+                    ldmatrix_x4(b_off(nt) + slot * b_slot(nt) + b_col(nt, h2), B);
+                    bf[2 * h2][nt][0] = B[0];
+                    bf[2 * h2][nt][1] = B[1];
+                    bf[2 * h2 + 1][nt][0] = B[2];
+                    bf[2 * h2 + 1][nt][1] = B[3];
+                }
             if constexpr (FAST) {
                 if (rs >= g_next) advance_group();
 #pragma unroll
@@ -431,8 +458,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            mma_chunk(c, R[c][2 * hh], R[c][2 * hh + 1], bf[2 * q + hh][0], bf[2 * q + hh][1]);
+                        for (int c = 0; c < 4; ++c) mma_chunk(c, R[c][2 * hh], R[c][2 * hh + 1], 2 * q + hh);
                 }
             } else {
 #pragma unroll
@@ -445,7 +471,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
                     for (int c = 0; c < 4; ++c) {
                         uint32_t x0, x1;
                         ldmatrix_x2_trans(wst + row * 64 + 16 * (c ^ ((row >> 1) & 3)), x0, x1);
-                        mma_chunk(c, x0, x1, bf[h][0], bf[h][1]);
+                        mma_chunk(c, x0, x1, h);
                     }
                 }
             }
@@ -468,9 +494,11 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
                 const int m = item / kTileN, nl = item % kTileN;
                 const int64_t n = (int64_t)tile * kTileN + nl;
-                // (m, nl) is entry i = 2 (nl % 4) + (m % 2) of chunk nl / 32 at lane 4 ((nl % 32) / 4) + m / 2
-                const int i = 2 * (nl & 3) + (m & 1);
-                const int src = 32 * ((nl >> 5) * NI + (MT > 1 ? i : i / 2)) + 4 * ((nl & 31) >> 2) + (m >> 1);
+                // (m, nl) is entry i = 2 (nl % 4) + (m % 2) of batch tile m / 8 of chunk nl / 32, held by
+                // lane 4 ((nl % 32) / 4) + (m % 8) / 2
+                const int mm = m & 7, i = 2 * (nl & 3) + (mm & 1);
+                const int src = 32 * ((nl >> 5) * NI + (m >> 3) * NB + (MT > 1 ? i : i / 2)) + 4 * ((nl & 31) >> 2) +
+                                (mm >> 1);
                 float v = 0.f;
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) v += tots[w * 4 * NI * 32 + src];
@@ -531,13 +559,21 @@ SkFn select_sk_t(int mt) {
         case 5: return gemv_sk_kernel<5, FAST>;
         case 6: return gemv_sk_kernel<6, FAST>;
         case 7: return gemv_sk_kernel<7, FAST>;
-        default: return gemv_sk_kernel<8, FAST>;
+        case 8: return gemv_sk_kernel<8, FAST>;
+        case 9: return gemv_sk_kernel<9, FAST>;
+        case 10: return gemv_sk_kernel<10, FAST>;
+        case 11: return gemv_sk_kernel<11, FAST>;
+        case 12: return gemv_sk_kernel<12, FAST>;
+        case 13: return gemv_sk_kernel<13, FAST>;
+        case 14: return gemv_sk_kernel<14, FAST>;
+        case 15: return gemv_sk_kernel<15, FAST>;
+        default: return gemv_sk_kernel<16, FAST>;
     }
 }
 // Occupancy queries use the FAST instance (both have the same shared memory and launch bounds).
 SkFn select_sk(int mt, bool fast = true) { return fast ? select_sk_t<true>(mt) : select_sk_t<false>(mt); }
 
-std::atomic<int> g_sk_occ[9];
+std::atomic<int> g_sk_occ[kMaxMT + 1];
 
 // Resident CTAs per SM from the kernel's registers and shared memory.
 int sk_ctas_per_sm(int mt) {
@@ -558,7 +594,7 @@ int sk_ctas_per_sm(int mt) {
     return n;
 }
 
-std::atomic<int> g_sk_clusters[9][kMaxCluster + 1];
+std::atomic<int> g_sk_clusters[kMaxMT + 1][kMaxCluster + 1];
 
 // Clusters of S CTAs that can be resident at once (clusters are placed within one GPC each, so
 // this can be less than the resident CTAs divided by S).
@@ -588,34 +624,23 @@ int sk_max_clusters(int mt, int S) {
     return n;
 }
 
-}  // namespace
-
-bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s) {
-    const int64_t units = (N + kTileN - 1) / kTileN * ((K + kRows - 1) / kRows);   // counted in 32 bits
-    return N % 32 == 0 && units < ((int64_t)1 << 31) && (reinterpret_cast<uintptr_t>(b) % 16) == 0 &&
-           (reinterpret_cast<uintptr_t>(a) % 16) == 0 && (reinterpret_cast<uintptr_t>(s) % 8) == 0;
-}
-
-GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count) {
-    (void)G;
-    GemvPlan pl{};
-    pl.tma = true;
-    pl.mma = true;
-    pl.vec = 1;
-    pl.m_rows = (int)std::min<int64_t>(M, 8);
-    pl.col_tiles = (int)((N + kTileN - 1) / kTileN);
-    const int64_t T = pl.col_tiles, nblk = (K + kRows - 1) / kRows;
+// Cluster layout of one launch of mt activation rows: S CTAs per cluster over k whole tiles each,
+// all resident at once; the fewest units per CTA wins, then the most CTAs. An explicit split asks
+// for that many CTAs per tile (at most a cluster, at most one per unit).
+struct SkLayout {
+    int cluster, cluster_tiles, ctas;
+    int64_t nblk;
+};
+SkLayout sk_layout(int mt, int64_t N, int64_t K, int split_k_request, int sm_count) {
+    const int64_t T = (N + kTileN - 1) / kTileN, nblk = (K + rows_for(mt) - 1) / rows_for(mt);
     int best_s = 1, best_k = 1;
     if (split_k_request > 0) {
-        // That many CTAs per tile (at most a cluster, at most one per unit).
         best_s = (int)std::min<int64_t>(std::min(split_k_request, kMaxCluster), nblk);
     } else {
-        // Clusters of S CTAs over k whole tiles each, all resident at once: the fewest units per
-        // CTA wins, then the most CTAs.
-        const int64_t slots = (int64_t)std::max(sm_count, 1) * sk_ctas_per_sm(pl.m_rows);
+        const int64_t slots = (int64_t)std::max(sm_count, 1) * sk_ctas_per_sm(mt);
         int64_t best_cost = INT64_MAX, best_ctas = 0;
         for (int S = 1; S <= kMaxCluster; ++S) {
-            const int64_t qmax = std::min<int64_t>({T, slots / S, (int64_t)sk_max_clusters(pl.m_rows, S)});
+            const int64_t qmax = std::min<int64_t>({T, slots / S, (int64_t)sk_max_clusters(mt, S)});
             for (int64_t Q = 1; Q <= qmax; ++Q) {
                 const int64_t k = (T + Q - 1) / Q;
                 if ((Q - 1) * k >= T) continue;   // the same k with fewer clusters
@@ -631,9 +656,35 @@ GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_r
             }
         }
     }
-    pl.cluster = best_s;
-    pl.cluster_tiles = best_k;
-    pl.split_k = (int)((T + best_k - 1) / best_k) * best_s;  // the grid size
+    SkLayout l;
+    l.cluster = best_s;
+    l.cluster_tiles = best_k;
+    l.ctas = (int)((T + best_k - 1) / best_k) * best_s;
+    l.nblk = nblk;
+    return l;
+}
+
+}  // namespace
+
+bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s) {
+    const int64_t units = (N + kTileN - 1) / kTileN * ((K + 63) / 64);   // counted in 32 bits (64-row units at most)
+    return N % 32 == 0 && units < ((int64_t)1 << 31) && (reinterpret_cast<uintptr_t>(b) % 16) == 0 &&
+           (reinterpret_cast<uintptr_t>(a) % 16) == 0 && (reinterpret_cast<uintptr_t>(s) % 8) == 0;
+}
+
+GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count) {
+    (void)G;
+    GemvPlan pl{};
+    pl.tma = true;
+    pl.mma = true;
+    pl.vec = 1;
+    pl.m_rows = (int)std::min<int64_t>(M, kMaxMT);
+    pl.col_tiles = (int)((N + kTileN - 1) / kTileN);
+    const SkLayout l = sk_layout(pl.m_rows, N, K, split_k_request, sm_count);
+    pl.cluster = l.cluster;
+    pl.cluster_tiles = l.cluster_tiles;
+    pl.split_k = l.ctas;
+    pl.split_k_request = split_k_request;
     pl.ws_bytes = 0;  // partial sums stay in the clusters' shared memory
     return pl;
 }
@@ -641,29 +692,36 @@ GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_r
 cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M,
                             int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace,
                             const GemvPlan& pl, const WaitPolicy& wp, cudaStream_t st) {
-    CUtensorMap bmap;
-    {
-        const cuuint64_t dims[2] = {(cuuint64_t)(N / 8), (cuuint64_t)K};
-        const cuuint64_t strides[1] = {(cuuint64_t)(N / 8) * 4};
-        const cuuint32_t box[2] = {(cuuint32_t)kTileWords, (cuuint32_t)kRows};
-        const cuuint32_t estr[2] = {1, 1};
-        cudaError_t e = encode_tensor_map(&bmap, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, (void*)b, dims, strides, box,
-                                          estr, CU_TENSOR_MAP_SWIZZLE_64B);
-        if (e != cudaSuccess) return e;
-    }
-    const int64_t nblk = (K + kRows - 1) / kRows;
     char* ws = static_cast<char*>(workspace);
-    for (int64_t m0 = 0; m0 < M; m0 += 8) {
-        const int mt = (int)std::min<int64_t>(8, M - m0);
-        CUtensorMap amap;
-        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)mt};
-        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)kRows, (cuuint32_t)mt};
-        const cuuint32_t estr[2] = {1, 1};
-        cudaError_t e = encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)(a + m0 * K), dims,
-                                          strides, box, estr,
-                                          a_swizzled(mt) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
-        if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int split_req = pl.split_k_request;
+    for (int64_t m0 = 0; m0 < M; m0 += kMaxMT) {
+        const int mt = (int)std::min<int64_t>(kMaxMT, M - m0);
+        const int rows = rows_for(mt);
+        // Row blocks of another size than the first take their own layout (stage rows differ).
+        const SkLayout l = mt == pl.m_rows ? SkLayout{pl.cluster, pl.cluster_tiles, pl.split_k, (K + rows - 1) / rows}
+                                           : sk_layout(mt, N, K, split_req, sms);
+        CUtensorMap bmap, amap;
+        {
+            const cuuint64_t dims[2] = {(cuuint64_t)(N / 8), (cuuint64_t)K};
+            const cuuint64_t strides[1] = {(cuuint64_t)(N / 8) * 4};
+            const cuuint32_t box[2] = {(cuuint32_t)kTileWords, (cuuint32_t)rows};
+            const cuuint32_t estr[2] = {1, 1};
+            cudaError_t e = encode_tensor_map(&bmap, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, (void*)b, dims, strides, box,
+                                              estr, CU_TENSOR_MAP_SWIZZLE_64B);
+            if (e != cudaSuccess) return e;
+        }
+        {
+            const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)mt};
+            const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+            const cuuint32_t box[2] = {(cuuint32_t)rows, (cuuint32_t)mt};
+            const cuuint32_t estr[2] = {1, 1};
+            cudaError_t e = encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)(a + m0 * K), dims,
+                                              strides, box, estr,
+                                              a_swizzled(mt) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+            if (e != cudaSuccess) return e;
+        }
         SkArgs args;
         args.s = s;
         args.z = z;
@@ -672,25 +730,25 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         args.N = N;
         args.K = K;
         args.tiles = pl.col_tiles;
-        args.tiles_per_cluster = pl.cluster_tiles;
+        args.tiles_per_cluster = l.cluster_tiles;
         args.G = G;
         args.zp_bias = zp_bias;
-        args.nblk = (int)nblk;
+        args.nblk = (int)l.nblk;
         args.magic = kMagic;
         args.stall_loads = wp.stall_loads;
         args.wait_ns = wp.limit_ns;
         const size_t smem = sk_smem_bytes(mt);
-        SkFn k = select_sk(mt, G % kRows == 0);
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        SkFn k = select_sk(mt, G % rows == 0);
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg{};
-        cfg.gridDim = dim3((unsigned)pl.split_k);
+        cfg.gridDim = dim3((unsigned)l.ctas);
         cfg.blockDim = dim3(kThreads);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)pl.cluster;
+        attr[0].val.clusterDim.x = (unsigned)l.cluster;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
