@@ -172,8 +172,8 @@ class Problem:
                           workspace=self.ws, stream=stream, pdl=self.pdl)
 
     def launches_per_step(self):
-        # GEMV for M <= 8; tensor-core GEMM (one launch per 128 rows) above.
-        return 1 if self.M <= 8 else (self.M + 127) // 128
+        # GEMV (one launch per 16 rows) for M <= 32; tensor-core GEMM (one per 128 rows) above.
+        return (self.M + 15) // 16 if self.M <= 32 else (self.M + 127) // 128
 
 
 def copies_for(bytes_per_copy):
@@ -217,7 +217,7 @@ def measure_problem(torch, prob, steps_per_graph, reps):
 def summary(prob, per_step_s, peaks, tensor_bound):
     gbs = prob.bytes / per_step_s / 1e9
     tfs = prob.flops / per_step_s / 1e12
-    # every path multiplies on the tensor cores (mma.sync for M <= 8, tcgen05 above)
+    # every path multiplies on the tensor cores (mma.sync for M <= 32, tcgen05 above)
     t_hbm = prob.bytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = prob.flops / (peaks["bf16_tflops"] * 1e12)
     t_roof = max(t_hbm, t_tc)
@@ -337,8 +337,8 @@ def run_gpu(args):
     Problem.pdl = args.pdl
     achieved = prob.bytes / per_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
-    kernel_name = "tc_gemm_kernel<32>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
-    traffic = traffic_from_profiles("tc_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
+    kernel_name = "gemv_sk_kernel<16, true>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
+    traffic = traffic_from_profiles("gemv_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
 
     extras = {}
     if rank == 0 and not args.no_extras:

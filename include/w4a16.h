@@ -98,8 +98,9 @@ W4A16_API size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int
  *             symmetric form, where every zero point is zp_bias. When qzeros is
  *             given, zp_bias is ignored.
  *   M, N, K   M >= 1, N >= 8, K >= group_size; N % 8 == 0; K % group_size == 0.
- *             M <= 16 runs the GEMV (warp mma.sync); M > 16 the tcgen05
- *             tensor-core GEMM when its shape and alignment rules hold.
+ *             M <= 32 runs the GEMV (warp mma.sync, one launch per 16 rows);
+ *             M > 32 the tcgen05 tensor-core GEMM when its shape and
+ *             alignment rules hold.
  *   group_size G: G >= 16 and G % 16 == 0.
  *   zp_bias   0..15 when qzeros is NULL.
  *   out       fp16 [M, N], device, 2-byte aligned; fully overwritten; must not
@@ -126,7 +127,7 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
 /*
  * Kernel selection for tests and measurement.
  *   kernel: W4A16_KERNEL_AUTO uses the same table as w4a16_gemm (GEMV for
- *     M <= 16, tensor cores for M > 16 when N % 128 == 0, K % 64 == 0 and a,
+ *     M <= 32, tensor cores for M > 32 when N % 128 == 0, K % 64 == 0 and a,
  *     b_packed are 16-byte aligned); GEMV forces the GEMV family (any M; larger
  *     M runs it once per block of 16 rows of A): its multiply-accumulate uses
  *     warp mma.sync when N % 32 == 0, a and b_packed are 16-byte and scales
