@@ -339,6 +339,8 @@ def run_gpu(args):
     hbm_peak = float(peaks["hbm_gbs"])
     kernel_name = "gemv_sk_kernel<16, true>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
     traffic = traffic_from_profiles("gemv_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
+    if traffic is not None:  # per step, like `achieved` (the batch-32 step is two 16-row launches)
+        traffic = traffic * prob.launches_per_step()
 
     extras = {}
     if rank == 0 and not args.no_extras:
