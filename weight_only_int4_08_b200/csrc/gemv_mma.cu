@@ -65,7 +65,14 @@ constexpr int kTileWords = kTileN / 8;            // 16 packed words = 64 B per 
 #define W4A16_SK_RING 2
 #endif
 constexpr int kRing = W4A16_SK_RING;              // stages in flight per warp
-constexpr int kMaxCluster = 8;                    // portable thread-block cluster size
+#ifndef W4A16_SK_MAX_CLUSTER
+#define W4A16_SK_MAX_CLUSTER 4
+#endif
+// Thread-block cluster size limit (above 8: non-portable). Measured on B200 over the decode,
+// small-batch and layer shapes: a limit of 4 was as fast as or faster than 8 on every shape
+// (K=4096, N=6144: 9.6 -> 8.1 us) and 16 was slower; clusters cost more than the finer
+// split they buy.
+constexpr int kMaxCluster = W4A16_SK_MAX_CLUSTER;
 constexpr int kMaxMT = 16;                        // activation rows per launch: two 8-row MMA tiles
 
 // MMA batch tiles (8 activation rows each) of a launch of MT rows.
@@ -604,6 +611,7 @@ int sk_max_clusters(int mt, int S) {
     SkFn k = select_sk(mt);
     const size_t smem = sk_smem_bytes(mt);
     n = 0;
+    if (kMaxCluster > 8) cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3((unsigned)S);
@@ -741,6 +749,10 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         SkFn k = select_sk(mt, G % rows == 0);
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
+        if (l.cluster > 8) {
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+        }
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3((unsigned)l.ctas);
         cfg.blockDim = dim3(kThreads);
