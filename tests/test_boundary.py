@@ -106,6 +106,23 @@ def test_options_are_checked():
     o = w.W4A16Options(1, 999)
     rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
     assert rc == w.W4A16_ERR_INVALID_ARG
+    o = w.W4A16Options(0, 0, 0, 0, 2)   # an undefined launch flag
+    rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
+    assert rc == w.W4A16_ERR_INVALID_ARG
+    assert "launch flag" in w.lib.w4a16_last_error().decode()
+    o = w.W4A16Options(0, 0, 4, 0, 0)   # an undefined debug flag
+    rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
+    assert rc == w.W4A16_ERR_INVALID_ARG
+
+
+def test_options_struct_matches_the_header():
+    # field names and order of w4a16_gemm_options as include/w4a16.h declares them
+
+    hdr = open(os.path.join(ROOT, "include", "w4a16.h")).read()
+    body = re.search(r"typedef struct \{(.*?)\} w4a16_gemm_options;", hdr, re.S).group(1)
+    fields = re.findall(r"(?:int32_t|uint32_t)\s+(\w+);", body)
+    assert fields == [f for f, _ in w.W4A16Options._fields_]
+    assert ctypes.sizeof(w.W4A16Options) == 4 * len(fields)
 
 
 def test_workspace_query_rejects_bad_shapes():
