@@ -117,7 +117,6 @@ def test_options_are_checked():
 
 def test_options_struct_matches_the_header():
     # field names and order of w4a16_gemm_options as include/w4a16.h declares them
-
     hdr = open(os.path.join(ROOT, "include", "w4a16.h")).read()
     body = re.search(r"typedef struct \{(.*?)\} w4a16_gemm_options;", hdr, re.S).group(1)
     fields = re.findall(r"(?:int32_t|uint32_t)\s+(\w+);", body)
