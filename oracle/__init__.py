@@ -55,6 +55,10 @@ def load(path: str):
     L.oracle_repack.restype = ctypes.c_int
     L.oracle_unrepack.argtypes = [p, i64, i64, p]
     L.oracle_unrepack.restype = ctypes.c_int
+    L.oracle_ct_scales.argtypes = [p, i64, i64, p]
+    L.oracle_ct_scales.restype = ctypes.c_int
+    L.oracle_ct_zeros.argtypes = [p, i64, i64, p]
+    L.oracle_ct_zeros.restype = ctypes.c_int
     L.oracle_gemm_cols.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, i64, p, p]
     L.oracle_gemm_cols.restype = ctypes.c_int
     L.oracle_gemm.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p]
@@ -133,6 +137,28 @@ def unrepack(b: np.ndarray, K: int, N: int) -> np.ndarray:
     rc = lib().oracle_unrepack(_ptr(b), K, N, _ptr(out))
     if rc:
         raise ValueError(f"oracle_unrepack failed ({rc})")
+    return out
+
+
+def ct_scales(s_ng: np.ndarray, N: int, ngroups: int) -> np.ndarray:
+    """Checkpoint scales [N, K/G] -> kernel scales [K/G, N] (fp16 bits as uint16)."""
+    s_ng = _c(s_ng, np.uint16)
+    assert s_ng.size == N * ngroups
+    out = np.empty((ngroups, N), np.uint16)
+    rc = lib().oracle_ct_scales(_ptr(s_ng), N, ngroups, _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_ct_scales failed ({rc})")
+    return out
+
+
+def ct_zeros(z_n8g: np.ndarray, N: int, ngroups: int) -> np.ndarray:
+    """Checkpoint zeros [N/8, K/G] -> kernel zeros [K/G, N/8] (uint32)."""
+    z_n8g = _c(z_n8g, np.uint32)
+    assert z_n8g.size == (N // 8) * ngroups
+    out = np.empty((ngroups, N // 8), np.uint32)
+    rc = lib().oracle_ct_zeros(_ptr(z_n8g), N, ngroups, _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_ct_zeros failed ({rc})")
     return out
 
 

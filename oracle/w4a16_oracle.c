@@ -165,6 +165,42 @@ int oracle_unrepack(const uint32_t* b, int64_t K, int64_t N, uint32_t* ckpt)
     return 0;
 }
 
+/* ---------------- checkpoint scales and zeros -> kernel layout ----------------
+ * Section "2. 가중치 레이아웃 재포장 (Weight Repacking)" of the PR #37352 page
+ * states the layer's layout after loading: weight [K, N/8] and scale [K/G, N].
+ * The checkpoint side of the scales and zeros is a reading (the page prints only
+ * the weight's): scales are stored per output channel, [N, K/G] fp16 with
+ * element (n, g) at n * (K/G) + g; zeros are packed 8 output channels per int32
+ * like the kernel's zeros, [N/8, K/G], word (c, g) holding z[8c + j][g] in
+ * nibble j. The kernel zeros are [K/G, N/8], word (g, d) holding z[g][8d + j].
+ * ngroups = K / G. Both conversions move values only: bit-exact. */
+int oracle_ct_scales(const uint16_t* s_ng, int64_t N, int64_t ngroups, uint16_t* s_gn)
+{
+    if (N <= 0 || ngroups <= 0) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < ngroups; ++g)
+            s_gn[g * N + n] = s_ng[n * ngroups + g];
+    return 0;
+}
+
+int oracle_ct_zeros(const uint32_t* z_n8g, int64_t N, int64_t ngroups, uint32_t* z_gn8)
+{
+    if (N <= 0 || ngroups <= 0 || N % 8) return -1;
+    uint8_t* z = (uint8_t*)malloc((size_t)(N * ngroups));   /* z[n][g], one nibble per byte */
+    if (!z) return -2;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < ngroups; ++g)
+            z[n * ngroups + g] = nibble(z_n8g[(n / 8) * ngroups + g], (int)(n % 8));
+    for (int64_t g = 0; g < ngroups; ++g)
+        for (int64_t d = 0; d < N / 8; ++d) {
+            uint32_t word = 0;
+            for (int j = 0; j < 8; ++j) word |= (uint32_t)z[(8 * d + j) * ngroups + g] << (4 * j);
+            z_gn8[g * (N / 8) + d] = word;
+        }
+    free(z);
+    return 0;
+}
+
 /* ---------------- GEMM ---------------------------------------------------
  * a      fp16 bits [M, K]
  * b      packed    [K, N/8]

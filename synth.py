@@ -20,7 +20,7 @@ from __future__ import annotations
 import numpy as np
 
 # tensor ids: one stream each
-T_A, T_B, T_S, T_Z, T_CKPT = 1, 2, 3, 4, 5
+T_A, T_B, T_S, T_Z, T_CKPT, T_CT_S, T_CT_Z = 1, 2, 3, 4, 5, 6, 7
 
 
 def rng(seed: int, tensor_id: int, layer: int = 0) -> np.random.Generator:
@@ -68,6 +68,16 @@ def make_case(M, K, N, G, *, sym: bool, seed: int, a_dist: str = "normal",
     case["s"] = fp16_uniform(rng(seed, T_S, layer), (K // G, N), s_lo, s_hi)
     case["z"] = None if sym else words_nibbles_in(rng(seed, T_Z, layer), (K // G, N // 8), z_lo, z_hi)
     return case
+
+
+def ct_checkpoint(K, N, G, *, sym: bool, seed: int, s_lo: float = 0.002, s_hi: float = 0.02,
+                  z_lo: int = 6, z_hi: int = 10):
+    """A layer as the checkpoint stores it: weight [N, K/8], scales [N, K/G] fp16 and,
+    unless sym, zeros [N/8, K/G] (8 output channels per int32)."""
+    return dict(K=K, N=N, G=G, sym=sym, seed=seed,
+                ckpt=words_uniform(rng(seed, T_CKPT), (N, K // 8)),
+                s_ng=fp16_uniform(rng(seed, T_CT_S), (N, K // G), s_lo, s_hi),
+                z_n8g=None if sym else words_nibbles_in(rng(seed, T_CT_Z), (N // 8, K // G), z_lo, z_hi))
 
 
 # ---- the five workloads -----------------------------------------------------

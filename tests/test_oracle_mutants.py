@@ -28,6 +28,11 @@ MUTANTS = {
                       "int zz = zp_bias;"),
     "round_half_down": ("if (rem > halfway || (rem == halfway && (keep & 1))) keep += 1;",
                         "if (rem > halfway) keep += 1;"),
+    "ct_zero_nibble": ("z[n * ngroups + g] = nibble(z_n8g[(n / 8) * ngroups + g], (int)(n % 8));",
+                       "z[n * ngroups + g] = nibble(z_n8g[(n / 8) * ngroups + g], (int)(7 - n % 8));"),
+    "ct_zero_word": ("z[n * ngroups + g] = nibble(z_n8g[(n / 8) * ngroups + g], (int)(n % 8));",
+                     "z[n * ngroups + g] = nibble(z_n8g[(n / 8) + g * (N / 8)], (int)(n % 8));"),
+    "ct_scales_untransposed": ("s_gn[g * N + n] = s_ng[n * ngroups + g];", "s_gn[g * N + n] = s_ng[g * N + n];"),
     "scale_of_wrong_group": ("float sc = oracle_half_to_float(s[g * N + n]);",
                              "float sc = oracle_half_to_float(s[n]);"),
 }
@@ -44,6 +49,10 @@ def _pins():
     yield "q_eq_z", T.test_q_equals_z_gives_zero
     yield "integer_matmul", T.test_integer_matmul_special_case
     yield "repack_single", T.test_repack_tracks_every_single_nibble
+    yield "worked_ct_load", lambda: T.test_worked_ct_load(g)
+    yield "ct_single", T.test_ct_load_tracks_every_single_element
+    for sym in (True, False):
+        yield f"ct_dense{sym}", (lambda s=sym: T.test_ct_load_preserves_the_dequantised_weight(s))
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
