@@ -389,7 +389,7 @@ def run_gpu(args):
 
 
 def run_extras(torch, w, peaks):
-    """The other workloads: small-batch sweep, batch-32 with repack, 32-layer stack."""
+    """The other workloads: small-batch sweep, batch-32 with repack (and the whole-layer load), 32-layer stack."""
     ex = {}
     for M in (1, 2, 4, 8, 16):
         c = synth.config3(M)
@@ -413,11 +413,34 @@ def run_extras(torch, w, peaks):
     ex["config4_repack"] = {"us": round(per * 1e6, 3), "GB/s": round(rbytes / per / 1e9, 1),
                             "frac_of_roofline": round(rbytes / (peaks["hbm_gbs"] * 1e9) / per, 4)}
     del cks, outs
+    ex["config4_load_ct"] = measure_load_ct(torch, w, peaks)
     p = Problem(w, torch, c, copies_for(alg_bytes(32, 4096, 14336, 128, True)), b=bkn)
     ex["config4_M32"] = summary(p, measure_problem(torch, p, 16, 20), peaks, tensor_bound=True)
     del p
     ex.update(run_stack(torch, w, peaks))
     return ex
+
+
+def measure_load_ct(torch, w, peaks):
+    """The batch-32 workload's layer loaded from the checkpoint layout (weight, scales, zeros) in one launch;
+    four copies rotate so every call reads and writes 30 MB that are not in L2."""
+    K, N, G = 4096, 14336, 128
+    c = synth.ct_checkpoint(K, N, G, sym=False, seed=3)
+    ins = [(to_dev(c["ckpt"], torch), to_dev(c["s_ng"], torch), to_dev(c["z_n8g"], torch)) for _ in range(4)]
+    outs = [(torch.empty((K, N // 8), dtype=torch.int32, device="cuda"),
+             torch.empty((K // G, N), dtype=torch.float16, device="cuda"),
+             torch.empty((K // G, N // 8), dtype=torch.int32, device="cuda")) for _ in range(4)]
+    state = {"i": 0}
+
+    def ld():
+        j = state["i"] % 4
+        state["i"] += 1
+        w.w4a16_load_ct(*ins[j], N, K, G, out=outs[j])
+
+    per = measure_problem(torch, type("P", (), {"step": staticmethod(ld)})(), 16, 10)
+    nbytes = 2 * (N * K // 2 + N * (K // G) * 2 + (N // 8) * (K // G) * 4)   # read + write of each tensor
+    return {"us": round(per * 1e6, 3), "GB/s": round(nbytes / per / 1e9, 1),
+            "frac_of_roofline": round(nbytes / (peaks["hbm_gbs"] * 1e9) / per, 4)}
 
 
 def run_stack(torch, w, peaks):

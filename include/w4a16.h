@@ -76,6 +76,36 @@ typedef enum {
 W4A16_API w4a16_status w4a16_repack(const void* ckpt_nk8, void* out_kn8, int64_t N, int64_t K, void* stream);
 
 /*
+ * w4a16_load_ct — a whole layer from the checkpoint layout to the kernel layout in
+ * one launch, bit-exact: the weight as w4a16_repack does it, the per-group scales
+ * [N, K/G] -> [K/G, N] and the packed zeros [N/8, K/G] -> [K/G, N/8].
+ *
+ * Cited operation: section "2. 가중치 레이아웃 재포장 (Weight Repacking)" of the
+ * PR #37352 analysis page: after loading, the layer's weight is [K, N//8] and its
+ * scale [K//G, N]. The page gives the checkpoint layout of the weight only; the
+ * scale and zero layouts on the checkpoint side are read as one row per output
+ * channel (scales) and 8 output channels per int32 (zeros, nibble j of word
+ * (c, g) = zero of channel 8c + j in group g, the kernel zeros' packing).
+ *
+ *   ckpt_nk8     const int32 [N, K/8], device, 4-byte aligned.
+ *   scale_ng     const fp16 [N, K/G], device, 2-byte aligned.
+ *   zero_n8g     const int32 [N/8, K/G], device, 4-byte aligned; or NULL for a
+ *                symmetric layer (then zero_gn8 is not written and may be NULL).
+ *   N, K, group_size  the w4a16_gemm shape rules for N, K and G.
+ *   out_kn8      int32 [K, N/8], device, 4-byte aligned; fully overwritten.
+ *   scale_gn     fp16 [K/G, N], device, 2-byte aligned; fully overwritten.
+ *   zero_gn8     int32 [K/G, N/8], device, 4-byte aligned; fully overwritten
+ *                when zero_n8g is given.
+ *   stream       cudaStream_t as void*.
+ * No output may overlap any input or another output.
+ * Errors: INVALID_ARG for a NULL pointer, a size rule broken, misalignment or
+ * overlapping buffers; UNSUPPORTED off sm_100; CUDA for a launch failure.
+ */
+W4A16_API w4a16_status w4a16_load_ct(const void* ckpt_nk8, const void* scale_ng, const void* zero_n8g, int64_t N,
+                                     int64_t K, int32_t group_size, void* out_kn8, void* scale_gn, void* zero_gn8,
+                                     void* stream);
+
+/*
  * w4a16_gemm_workspace_bytes — bytes of device workspace w4a16_gemm needs for
  * this shape on the current device (0 when the shape needs none). Returns 0 for
  * shapes w4a16_gemm would reject. The value depends on the current device's SM

@@ -23,7 +23,7 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     names = declared_symbols()
-    for required in ("w4a16_repack", "w4a16_gemm", "w4a16_gemm_workspace_bytes", "w4a16_status_string"):
+    for required in ("w4a16_repack", "w4a16_load_ct", "w4a16_gemm", "w4a16_gemm_workspace_bytes", "w4a16_status_string"):
         assert required in names
 
 
@@ -95,6 +95,27 @@ def test_repack_rejects_bad_arguments_on_host(kw, why):
     c = kw.get("c", P(0x1000))
     o = kw.get("o", P(0x80000000))
     rc = w.lib.w4a16_repack(c, o, kw.get("N", 64), kw.get("K", 64), None)
+    assert rc == w.W4A16_ERR_INVALID_ARG
+    assert why in w.lib.w4a16_last_error().decode()
+
+
+def load_ct(c=P(0x1000), s=P(0x2000000), z=None, N=64, K=256, G=128, o=P(0x80000000), so=P(0x90000000),
+            zo=None):
+    return w.lib.w4a16_load_ct(c, s, z, N, K, G, o, so, zo, None)
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(c=None), "NULL"), (dict(s=None), "NULL"), (dict(o=None), "NULL"), (dict(so=None), "NULL"),
+    (dict(z=P(0x3000000)), "zero_gn8"),
+    (dict(N=60), "N must be"), (dict(K=200), "K must be"), (dict(G=8, K=64), "group_size"),
+    (dict(c=P(0x1002)), "aligned"), (dict(s=P(0x2000001)), "aligned"), (dict(so=P(0x90000001)), "aligned"),
+    (dict(z=P(0x3000002), zo=P(0xA0000000)), "aligned"),
+    (dict(o=P(0x1000)), "overlaps an input"),            # weight out on the checkpoint weight
+    (dict(so=P(0x1000 + 64 * 256 // 2 - 2)), "overlaps an input"),   # scale out on the weight's last bytes
+    (dict(z=P(0x3000000), zo=P(0x90000000)), "outputs overlap"),     # zero out on the scale out
+])
+def test_load_ct_rejects_bad_arguments_on_host(kw, why):
+    rc = load_ct(**kw)
     assert rc == w.W4A16_ERR_INVALID_ARG
     assert why in w.lib.w4a16_last_error().decode()
 

@@ -37,6 +37,8 @@ LAUNCH_PDL = 1
 _p, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
 lib.w4a16_repack.argtypes = [_p, _p, _i64, _i64, _p]
 lib.w4a16_repack.restype = ctypes.c_int
+lib.w4a16_load_ct.argtypes = [_p, _p, _p, _i64, _i64, _i32, _p, _p, _p, _p]
+lib.w4a16_load_ct.restype = ctypes.c_int
 lib.w4a16_gemm_workspace_bytes.argtypes = [_i64, _i64, _i64, _i32]
 lib.w4a16_gemm_workspace_bytes.restype = _sz
 lib.w4a16_gemm_ex_workspace_bytes.argtypes = [_i64, _i64, _i64, _i32, ctypes.POINTER(W4A16Options)]
@@ -57,7 +59,7 @@ lib.w4a16_status_string.restype = ctypes.c_char_p
 lib.w4a16_last_error.argtypes = []
 lib.w4a16_last_error.restype = ctypes.c_char_p
 
-EXPORTED = ("w4a16_repack", "w4a16_gemm_workspace_bytes", "w4a16_gemm", "w4a16_gemm_ex_workspace_bytes",
+EXPORTED = ("w4a16_repack", "w4a16_load_ct", "w4a16_gemm_workspace_bytes", "w4a16_gemm", "w4a16_gemm_ex_workspace_bytes",
             "w4a16_gemm_ex", "w4a16_workspace_status", "w4a16_status_string", "w4a16_last_error",
             "w4a16_gemm_noalloc", "w4a16_noalloc_scratch_bytes")
 
@@ -126,6 +128,37 @@ def w4a16_repack(ckpt_nk8: torch.Tensor, N: int, K: int, out: torch.Tensor | Non
         raise ValueError("out must have N*K/8 elements")
     _check(lib.w4a16_repack(pc, po, N, K, _stream_ptr(stream)), "w4a16_repack")
     return out
+
+
+def w4a16_load_ct(ckpt_nk8: torch.Tensor, scale_ng: torch.Tensor, zero_n8g: torch.Tensor | None, N: int, K: int,
+                  group_size: int, out=None, stream=None):
+    """A checkpoint-layout layer -> the kernel layout in one launch (bit-exact).
+
+    ckpt_nk8 int32 [N, K/8], scale_ng fp16 [N, K/G], zero_n8g int32 [N/8, K/G] or None.
+    Returns (b_packed [K, N/8], scales [K/G, N], qzeros [K/G, N/8] or None); out, if
+    given, is such a tuple of preallocated tensors."""
+    G = group_size
+    ng = K // G if G > 0 else 0
+    pc = _dev(ckpt_nk8, "ckpt_nk8", (torch.int32, torch.uint32))
+    ps = _dev(scale_ng, "scale_ng", (torch.float16,))
+    pz = None if zero_n8g is None else _dev(zero_n8g, "zero_n8g", (torch.int32, torch.uint32))
+    if ckpt_nk8.numel() != N * K // 8 or scale_ng.numel() != N * ng:
+        raise ValueError("ckpt_nk8 must have N*K/8 elements and scale_ng N*(K/G)")
+    if zero_n8g is not None and zero_n8g.numel() != (N // 8) * ng:
+        raise ValueError("zero_n8g must have (N/8)*(K/G) elements")
+    dev = ckpt_nk8.device
+    if out is None:
+        out = (torch.empty((K, N // 8), dtype=torch.int32, device=dev),
+               torch.empty((ng, N), dtype=torch.float16, device=dev),
+               None if zero_n8g is None else torch.empty((ng, N // 8), dtype=torch.int32, device=dev))
+    b, s, z = out
+    pb = _dev(b, "out[0]", (torch.int32, torch.uint32))
+    pso = _dev(s, "out[1]", (torch.float16,))
+    pzo = None if z is None else _dev(z, "out[2]", (torch.int32, torch.uint32))
+    if b.numel() != N * K // 8 or s.numel() != N * ng or (z is not None and z.numel() != (N // 8) * ng):
+        raise ValueError("out tensors have the wrong sizes")
+    _check(lib.w4a16_load_ct(pc, ps, pz, N, K, G, pb, pso, pzo, _stream_ptr(stream)), "w4a16_load_ct")
+    return b, s, (z if zero_n8g is not None else None)
 
 
 def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qzeros: torch.Tensor | None,

@@ -85,6 +85,9 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
 
 cudaError_t launch_repack(const uint32_t* ckpt, uint32_t* out, int64_t N, int64_t K, cudaStream_t st);
 
+cudaError_t launch_ct_load(const uint32_t* ckpt, const uint16_t* s_ng, const uint32_t* z_n8g, uint32_t* b_kn8,
+                           uint16_t* s_gn, uint32_t* z_gn8, int64_t N, int64_t K, int64_t ngroups, cudaStream_t st);
+
 cudaError_t launch_gemv(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z,
                         int64_t M, int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out,
                         void* workspace, const GemvPlan& plan, const WaitPolicy& wp, cudaStream_t st);

@@ -1,4 +1,6 @@
-// Checkpoint [N, K/8] -> kernel [K, N/8] int4 weight repack (bit-exact).
+// Checkpoint [N, K/8] -> kernel [K, N/8] int4 weight repack (bit-exact), and the
+// whole-layer load conversion that also moves the per-group scales [N, K/G] ->
+// [K/G, N] and zeros [N/8, K/G] -> [K/G, N/8] in the same launch.
 //
 // Operation: section "2. 가중치 레이아웃 재포장 (Weight Repacking)" of the vLLM
 // PR #37352 analysis page. Checkpoint word (n, c) holds q[8c + j, n] in nibble j;
@@ -50,15 +52,15 @@ __device__ __forceinline__ void nibble_transpose8(uint32_t (&x)[8]) {
     }
 }
 
-__global__ void __launch_bounds__(kThreads)
-repack_kernel(const uint32_t* __restrict__ ckpt, uint32_t* __restrict__ out, int64_t N, int64_t K) {
-    __shared__ uint32_t tile[kTileRows * kTileWords];  // [k_local][n_word ^ swz]
+// One 256 (n) x 256 (k) tile of the weight repack; (bx, by) = (k-word tile, n tile).
+__device__ __forceinline__ void repack_tile(const uint32_t* __restrict__ ckpt, uint32_t* __restrict__ out, int64_t N,
+                                            int64_t K, int64_t bx, int64_t by, uint32_t* tile) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int64_t kw_total = K / 8;   // checkpoint words per row
     const int64_t nw_total = N / 8;   // kernel words per row
-    const int64_t kw0 = (int64_t)blockIdx.x * kTileWords;  // first checkpoint word column
-    const int64_t n0 = (int64_t)blockIdx.y * kTileRows;    // first n row
+    const int64_t kw0 = bx * kTileWords;  // first checkpoint word column
+    const int64_t n0 = by * kTileRows;    // first n row
 
     const int64_t kw = kw0 + lane;
     // Each warp transposes n-blocks b = warp, warp + 8, warp + 16, warp + 24.
@@ -90,6 +92,66 @@ repack_kernel(const uint32_t* __restrict__ ckpt, uint32_t* __restrict__ out, int
     }
 }
 
+__global__ void __launch_bounds__(kThreads)
+repack_kernel(const uint32_t* __restrict__ ckpt, uint32_t* __restrict__ out, int64_t N, int64_t K) {
+    __shared__ uint32_t tile[kTileRows * kTileWords];  // [k_local][n_word ^ swz]
+    repack_tile(ckpt, out, N, K, blockIdx.x, blockIdx.y, tile);
+}
+
+// out[c][r] = in[r][c] for one 32 x 32 tile (tr, tc) of an R x C matrix of T.
+// Lane = column on both sides, so loads and stores are row segments; the tile's
+// row pitch of 33 elements keeps the column reads of 32-bit T conflict free.
+template <typename T>
+__device__ __forceinline__ void transpose_tile(const T* __restrict__ in, T* __restrict__ out, int64_t R, int64_t C,
+                                               int64_t tr, int64_t tc, T* tile) {
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t r0 = tr * 32, c0 = tc * 32;
+#pragma unroll
+    for (int y = warp; y < 32; y += kThreads / 32) {
+        const int64_t r = r0 + y, c = c0 + lane;
+        if (r < R && c < C) tile[y * 33 + lane] = in[r * C + c];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int y = warp; y < 32; y += kThreads / 32) {
+        const int64_t c = c0 + y, r = r0 + lane;
+        if (r < R && c < C) out[c * R + r] = tile[lane * 33 + y];
+    }
+}
+
+struct CtLoadArgs {
+    const uint32_t* ckpt;   // [N, K/8]
+    const uint16_t* s_ng;   // [N, K/G]
+    const uint32_t* z_n8g;  // [N/8, K/G] or null
+    uint32_t* b_kn8;        // [K, N/8]
+    uint16_t* s_gn;         // [K/G, N]
+    uint32_t* z_gn8;        // [K/G, N/8] or null
+    int64_t N, K, ngroups;
+    int64_t rep_x, rep_blocks;   // weight tiles: x extent, count
+    int64_t s_tc, s_blocks;      // scale tiles: column-tile extent, count
+    int64_t z_tc;                // zero tiles: column-tile extent
+};
+
+// The whole layer in one launch: blocks [0, rep_blocks) repack weight tiles, the
+// next s_blocks transpose scale tiles, the rest transpose zero tiles.
+__global__ void __launch_bounds__(kThreads) ct_load_kernel(const CtLoadArgs p) {
+    __shared__ uint32_t smem[kTileRows * kTileWords];
+    int64_t b = blockIdx.x;
+    if (b < p.rep_blocks) {
+        repack_tile(p.ckpt, p.b_kn8, p.N, p.K, b % p.rep_x, b / p.rep_x, smem);
+        return;
+    }
+    b -= p.rep_blocks;
+    if (b < p.s_blocks) {
+        transpose_tile<uint16_t>(p.s_ng, p.s_gn, p.N, p.ngroups, b / p.s_tc, b % p.s_tc,
+                                 reinterpret_cast<uint16_t*>(smem));
+        return;
+    }
+    b -= p.s_blocks;
+    transpose_tile<uint32_t>(p.z_n8g, p.z_gn8, p.N / 8, p.ngroups, b / p.z_tc, b % p.z_tc, smem);
+}
+
 }  // namespace
 
 cudaError_t launch_repack(const uint32_t* ckpt, uint32_t* out, int64_t N, int64_t K, cudaStream_t st) {
@@ -97,6 +159,21 @@ cudaError_t launch_repack(const uint32_t* ckpt, uint32_t* out, int64_t N, int64_
     const int64_t gy = (N + kTileRows - 1) / kTileRows;
     if (gx > 0x7fffffff || gy > 65535) return cudaErrorInvalidValue;
     repack_kernel<<<dim3((unsigned)gx, (unsigned)gy), kThreads, 0, st>>>(ckpt, out, N, K);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ct_load(const uint32_t* ckpt, const uint16_t* s_ng, const uint32_t* z_n8g, uint32_t* b_kn8,
+                           uint16_t* s_gn, uint32_t* z_gn8, int64_t N, int64_t K, int64_t ngroups, cudaStream_t st) {
+    CtLoadArgs p{ckpt, s_ng, z_n8g, b_kn8, s_gn, z_gn8, N, K, ngroups, 0, 0, 0, 0, 0};
+    p.rep_x = (K / 8 + kTileWords - 1) / kTileWords;
+    p.rep_blocks = p.rep_x * ((N + kTileRows - 1) / kTileRows);
+    p.s_tc = (ngroups + 31) / 32;
+    p.s_blocks = p.s_tc * ((N + 31) / 32);
+    p.z_tc = p.s_tc;
+    const int64_t z_blocks = z_n8g ? p.z_tc * ((N / 8 + 31) / 32) : 0;
+    const int64_t blocks = p.rep_blocks + p.s_blocks + z_blocks;
+    if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
+    ct_load_kernel<<<(unsigned)blocks, kThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 

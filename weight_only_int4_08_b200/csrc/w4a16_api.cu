@@ -198,6 +198,42 @@ w4a16_status w4a16_repack(const void* ckpt_nk8, void* out_kn8, int64_t N, int64_
     return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
 }
 
+w4a16_status w4a16_load_ct(const void* ckpt_nk8, const void* scale_ng, const void* zero_n8g, int64_t N, int64_t K,
+                           int32_t group_size, void* out_kn8, void* scale_gn, void* zero_gn8, void* stream) {
+    g_last_error[0] = 0;
+    if (!ckpt_nk8 || !scale_ng || !out_kn8 || !scale_gn) return fail_arg("NULL pointer");
+    if (zero_n8g && !zero_gn8) return fail_arg("NULL pointer: zero_gn8 is needed when zero_n8g is given");
+    if (const char* why = check_gemm_shape(1, N, K, group_size)) return fail_arg(why);
+    if (!aligned(ckpt_nk8, 4) || !aligned(out_kn8, 4)) return fail_arg("weight pointers must be 4-byte aligned");
+    if (!aligned(scale_ng, 2) || !aligned(scale_gn, 2)) return fail_arg("scale pointers must be 2-byte aligned");
+    if (zero_n8g && (!aligned(zero_n8g, 4) || !aligned(zero_gn8, 4)))
+        return fail_arg("zero pointers must be 4-byte aligned");
+    const int64_t ng = K / group_size;
+    const size_t wb = (size_t)N * (size_t)K / 2, sb = (size_t)N * (size_t)ng * 2, zb = (size_t)N * (size_t)ng / 2;
+    const void* ins[3] = {ckpt_nk8, scale_ng, zero_n8g};
+    const size_t in_n[3] = {wb, sb, zb};
+    const void* outs[3] = {out_kn8, scale_gn, zero_n8g ? zero_gn8 : nullptr};
+    for (int i = 0; i < 3; ++i) {
+        if (!outs[i]) continue;
+        for (int j = 0; j < 3; ++j)
+            if (ins[j] && overlaps(outs[i], in_n[i], ins[j], in_n[j])) return fail_arg("an output overlaps an input");
+        for (int j = i + 1; j < 3; ++j)
+            if (outs[j] && overlaps(outs[i], in_n[i], outs[j], in_n[j])) return fail_arg("outputs overlap");
+    }
+    int sms = 0, maj = 0;
+    cudaError_t e = device_info(&sms, &maj);
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (maj != 10) {
+        set_error("unsupported: %s", "this library is built for sm_100 (B200) devices");
+        return W4A16_ERR_UNSUPPORTED;
+    }
+    e = launch_ct_load(static_cast<const uint32_t*>(ckpt_nk8), static_cast<const uint16_t*>(scale_ng),
+                       static_cast<const uint32_t*>(zero_n8g), static_cast<uint32_t*>(out_kn8),
+                       static_cast<uint16_t*>(scale_gn), zero_n8g ? static_cast<uint32_t*>(zero_gn8) : nullptr, N, K,
+                       ng, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
+}
+
 size_t w4a16_gemm_ex_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size,
                                      const w4a16_gemm_options* opts) {
     if (check_gemm_shape(M, N, K, group_size)) return 0;
