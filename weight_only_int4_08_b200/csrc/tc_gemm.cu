@@ -12,30 +12,39 @@
 // sum D_g is exact up to fp32 summation; the fp16 scale is applied in fp32 when
 // D_g is read back (tot += s[g, n] * D_g), never rounded into the weights.
 //
-// Roles (one CTA = one 128-column tile x one K slab; 10 warps):
-//   warp 4      producer: per stage of 64 k-rows, one 2-D TMA load of the
+// Roles (one CTA = one 128-column tile x one K slab; 14 warps, 10 above MN = 64;
+// the warp numbers below are those of the 14-warp form):
+//   warp 8      producer: per stage of 64 k-rows, one 2-D TMA load of the
 //               tile's packed words [64 rows x 64 B] (64-byte swizzle) and one of
 //               the activation tile [MN x 64] (128-byte swizzle, the canonical
-//               K-major layout of operand B);
-//   warps 0-3   dequantisers: warp p owns TMEM lanes 32p..32p+31 and tile
-//               columns 32p..32p+31 (one 16-byte chunk of each weight row);
-//               ldmatrix.trans hands every thread two k-rows of 4 columns per
-//               register, which become exact fp16 (q - z) pairs (0x6400 magic +
-//               fp16 subtract) written to TMEM with tcgen05.st.16x128b;
-//   warp 5      TMEM allocator and MMA issuer: tcgen05.mma.kind::f16 with A
+//               K-major layout of operand B), into an 8-stage ring;
+//   warps 0-7   dequantisers (0-3 above MN = 64): warp p owns TMEM lanes
+//               32(p%4)..+31 and tile columns 32(p%4)..+31 (one 16-byte chunk of
+//               each weight row); warps 0-3 take the even stages and 4-7 the odd
+//               ones; ldmatrix.trans hands every thread two k-rows of 4 columns
+//               per register, which become exact fp16 (q - z) pairs (0x6400 magic
+//               + fp16 subtract) written to TMEM with tcgen05.st.16x128b.x4;
+//   warp 9      TMEM allocator and MMA issuer: tcgen05.mma.kind::f16 with A
 //               from TMEM and B from shared memory, 4 per stage (K = 16 each);
 //               a fresh accumulator per group segment, double-buffered, and a
-//               tcgen05.commit to an mbarrier at each segment end;
-//   warps 6-9   epilogue: tcgen05.ld of each finished group segment, scaled by
+//               tcgen05.commit to an mbarrier at each segment end. When G is a
+//               multiple of 64 (segments are whole stages) the stage loop is
+//               unrolled over the ring so that every operand address is a
+//               constant offset: measured on B200, the issue loop's own
+//               instructions and barrier waits, not the tensor core, set the
+//               MMA rate at these small N (about 220 cycles per MMA with per-MMA
+//               bookkeeping, 62 with this form and one wait per stage, 36 for
+//               the MMAs alone at N = 32);
+//   warps 10-13 epilogue: tcgen05.ld of each finished group segment, scaled by
 //               s[g, n] in fp32 into register totals; then the fp16 output, or
 //               the fp32 split-K partial and the last-CTA ordered reduction.
 // Every mbarrier wait is bounded; a wait that runs out sets the workspace
 // status word to W4A16_ERR_TIMEOUT, and all roles drain and leave, freeing TMEM.
 //
-// Lane/column bookkeeping: dequantiser thread t of warp p (t0 = t % 4,
-// t1 = t / 4) holds tile columns 32p + 4 t1 + {0, 1, 2, 3} (nibbles 4(t1%2)..
-// of packed word 4p + t1/2) and writes them to TMEM lanes {t1, t1+8, t1+16,
-// t1+24} (+32p): lane L holds column 32p + 4 (L % 8) + L / 8. Columns at odd
+// Lane/column bookkeeping: dequantiser thread t of warp p (q = p % 4, t0 = t % 4,
+// t1 = t / 4) holds tile columns 32q + 4 t1 + {0, 1, 2, 3} (nibbles 4(t1%2)..
+// of packed word 4q + t1/2) and writes them to TMEM lanes {t1, t1+8, t1+16,
+// t1+24} (+32q): lane L holds column 32q + 4 (L % 8) + L / 8. Columns at odd
 // nibble positions come out of the unpack scaled by 16 (exact), undone in the
 // epilogue. The thread's k-pair in each 8-row matrix is t0, i.e. TMEM column
 // (k - k_stage) / 2 of the stage's A slot, in natural k order.
@@ -53,11 +62,16 @@ constexpr int kTileWords = kBlockN / 8;         // 16 packed words per k-row of 
 constexpr int kStageK = 64;                     // k-rows per pipeline stage
 constexpr int kWStageBytes = kStageK * kTileWords * 4;   // 64 rows x 64 B, 64-byte swizzle
 constexpr int kTmemStages = 4;                  // A slots in TMEM (32 columns = 64 k each)
-constexpr int kThreadsTC = 320;
+// Dequantiser warps: groups of four (one per TMEM lane quarter) that take turns on the stages,
+// two groups while the MMAs are short (MN <= 64), one above, where the per-column totals of
+// the epilogue need the registers that more threads would take. A group's stage ends with a
+// wait for its TMEM stores; a second group keeps another stage in flight meanwhile.
+__host__ __device__ constexpr int deq_warps(int mn) { return mn <= 64 ? 8 : 4; }
+__host__ __device__ constexpr int tc_threads(int mn) { return (deq_warps(mn) + 6) * 32; }
 
 template <int MN>
 struct TcCfg {
-    static constexpr int kSmemStages = MN <= 32 ? 8 : (MN <= 64 ? 6 : 4);
+    static constexpr int kSmemStages = 8;   // a multiple of kTmemStages (the unrolled issue loop relies on it)
     static constexpr int kBStageBytes = MN * 128;           // MN rows x 64 k x 2 B
     static constexpr int kDCol = kTmemStages * 32;          // first accumulator column
     static constexpr int kColsNeeded = kDCol + 2 * MN;
@@ -109,10 +123,13 @@ struct SegIter {
     int G;
 };
 
-template <int MN>
-__global__ void __launch_bounds__(kThreadsTC, (TcCfg<MN>::kTmemCols <= 256 && MN <= 32) ? 2 : 1)
+// FAST: G is a multiple of the 64-row stage, so group segments are whole stages.
+template <int MN, bool FAST>
+__global__ void __launch_bounds__(tc_threads(MN), (TcCfg<MN>::kTmemCols <= 256 && MN <= 32) ? 2 : 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap, TcArgs p) {
     using C = TcCfg<MN>;
+    constexpr int kDeqWarps = deq_warps(MN);
+    constexpr int kProducerWarp = kDeqWarps, kMmaWarp = kDeqWarps + 1, kEpiWarp0 = kDeqWarps + 2;
     constexpr int SS = C::kSmemStages;
     extern __shared__ __align__(1024) unsigned char s_raw[];
     unsigned char* s_base = reinterpret_cast<unsigned char*>(
@@ -141,7 +158,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             ptx::mbar_init(ptx::smem_addr(&bar_empty[i]), 1);
         }
         for (int i = 0; i < kTmemStages; ++i) {
-            ptx::mbar_init(ptx::smem_addr(&bar_afull[i]), 128);
+            ptx::mbar_init(ptx::smem_addr(&bar_afull[i]), 128);   // one group of four warps per stage
             ptx::mbar_init(ptx::smem_addr(&bar_aempty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -151,7 +168,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
         ptx::mbar_fence_init();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         ptx::tmem_alloc(ptx::smem_addr(&s_tmem), C::kTmemCols);
         ptx::tmem_relinquish();
     }
@@ -160,7 +177,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     ptx::tc_fence_after();
     const uint32_t tmem = s_tmem;
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
         // Converged loop, one elected lane issuing (as for the MMA warp).
         const bool leader = ptx::elect_one();
@@ -189,21 +206,42 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             for (int i = max(0, issued - SS); i < issued; ++i)
                 ptx::mbar_wait(ptx::smem_addr(&bar_full[i % SS]), (i / SS) & 1, &dummy, p.wait_ns);
         }
-    } else if (warp < 4) {
+    } else if (warp < kDeqWarps) {
         // -------------------------------------------------------- dequantisers
+        constexpr int kDeqGroups = kDeqWarps / 4;
+        const int q = warp & 3, dg = warp >> 2;   // TMEM lane quarter / column chunk; my group
         const int t1 = lane >> 2;
         const int64_t nw = p.N / 8;
-        const int64_t word = (int64_t)tile * kTileWords + 4 * warp + (t1 >> 1);  // holds my 4 columns
-        const int nib0 = 4 * (t1 & 1);                                           // their first nibble
+        const int64_t word = (int64_t)tile * kTileWords + 4 * q + (t1 >> 1);  // holds my 4 columns
+        const int nib0 = 4 * (t1 & 1);                                       // their first nibble
         const int64_t ngroups = p.K / p.G;
-        // Groups advance one at a time over the slab: g_cur is the open group, g_next_k its end.
-        int64_t g_cur = st_lo * kStageK / p.G - 1, g_next_k = (g_cur + 1) * p.G;
+        // g_next_k is the end of the open group. A warp that dequantises every other stage may skip
+        // groups, so the group is found from the row; its zero word is prefetched for the group
+        // after it.
+        int64_t g_next_k = st_lo * kStageK / p.G * p.G, g_pref = -1;
         uint32_t zw_next = 0u;
         bool have_next = false;
         uint32_t bias0 = 0, bias1 = 0, bias2 = 0, bias3 = 0;
         const uint32_t magic = p.magic;
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-        for (int i = 0; i < nst; ++i) {
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        auto enter_group = [&](int64_t kk) {
+            const int64_t g = kk / p.G;
+            g_next_k = (g + 1) * p.G;
+            uint32_t zraw = 0u;
+            if (p.z) {
+                zraw = have_next && g == g_pref ? zw_next : __ldg(p.z + g * nw + word);
+                g_pref = g + 1;
+                have_next = g_pref < ngroups;
+                if (have_next) zw_next = __ldg(p.z + g_pref * nw + word);
+            }
+            const uint32_t zw = p.z ? (zraw >> (4 * nib0)) : (uint32_t)p.zp_bias * 0x1111u;
+            // (1024 + z) for low-nibble columns, (1024 + 16 z) for high ones, in both halves
+            bias0 = (0x6400u + (zw & 0xFu)) * 0x00010001u;
+            bias1 = (0x6400u + 16u * ((zw >> 4) & 0xFu)) * 0x00010001u;
+            bias2 = (0x6400u + ((zw >> 8) & 0xFu)) * 0x00010001u;
+            bias3 = (0x6400u + 16u * ((zw >> 12) & 0xFu)) * 0x00010001u;
+        };
+        for (int i = dg; i < nst; i += kDeqGroups) {
             const int s = i % SS, ts = i % kTmemStages;
             // Wait outcomes are made warp-uniform: the tcgen05 stores below are .sync.aligned.
             bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns);
@@ -213,96 +251,138 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             ptx::tc_fence_after();
             const uint32_t wbase = ptx::smem_addr(s_w + (size_t)s * kWStageBytes);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                // rows 32h .. 32h + 31 as four 8x8 matrices of 16-bit halves; my address row
-                // is 32h + lane; 16-byte chunk `warp` of it, moved by the 64-byte swizzle
-                const int row = 32 * h + lane;
+            for (int hh = 0; hh < 2; ++hh) {
+                // rows 32hh .. 32hh + 31 as four 8x8 matrices of 16-bit halves; my address row is
+                // 32hh + lane; 16-byte chunk q of it, moved by the 64-byte swizzle
+                const int row = 32 * hh + lane;
                 uint32_t R[4];
-                ptx::ldmatrix_x4_trans(wbase + row * 64 + 16 * (warp ^ ((row >> 1) & 3)), R);
+                ptx::ldmatrix_x4_trans(wbase + row * 64 + 16 * (q ^ ((row >> 1) & 3)), R);
+                const int64_t k_half = (st_lo + i) * kStageK + 32 * hh;   // first k of this half stage
+                if (FAST && k_half >= g_next_k) enter_group(k_half);       // groups start at stage starts only
+                uint32_t lo[8], hi[8];
 #pragma unroll
                 for (int mi = 0; mi < 4; ++mi) {
-                    const int64_t kk = (st_lo + i) * kStageK + 32 * h + 8 * mi;   // first k of this matrix
-                    if (kk >= g_next_k) {   // G is a multiple of 16, so a group starts here or not at all
-                        const int64_t g = ++g_cur;
-                        g_next_k += p.G;
-                        // zero word of this group (prefetched one group ahead), then prefetch the next
-                        uint32_t zraw = 0u;
-                        if (p.z) {
-                            zraw = have_next ? zw_next : __ldg(p.z + g * nw + word);
-                            have_next = g + 1 < ngroups;
-                            if (have_next) zw_next = __ldg(p.z + (g + 1) * nw + word);
-                        }
-                        const uint32_t zw = p.z ? (zraw >> (4 * nib0)) : (uint32_t)p.zp_bias * 0x1111u;
-                        // (1024 + z) for low-nibble columns, (1024 + 16 z) for high ones, in both halves
-                        bias0 = (0x6400u + (zw & 0xFu)) * 0x00010001u;
-                        bias1 = (0x6400u + 16u * ((zw >> 4) & 0xFu)) * 0x00010001u;
-                        bias2 = (0x6400u + ((zw >> 8) & 0xFu)) * 0x00010001u;
-                        bias3 = (0x6400u + 16u * ((zw >> 12) & 0xFu)) * 0x00010001u;
-                    }
+                    // G % 16 == 0: an 8-row matrix never straddles a group boundary
+                    if (!FAST && k_half + 8 * mi >= g_next_k) enter_group(k_half + 8 * mi);
                     const uint32_t x = R[mi], y = x >> 8;
-                    const uint32_t col = (uint32_t)(ts * 32 + 16 * h + 4 * mi);
-                    ptx::tmem_st_16x128b(lane_base + col, hsub2((x & 0x000F000Fu) | magic, bias0),
-                                         hsub2((x & 0x00F000F0u) | magic, bias1));
-                    ptx::tmem_st_16x128b(lane_base + (16u << 16) + col, hsub2((y & 0x000F000Fu) | magic, bias2),
-                                         hsub2((y & 0x00F000F0u) | magic, bias3));
+                    lo[2 * mi] = hsub2((x & 0x000F000Fu) | magic, bias0);
+                    lo[2 * mi + 1] = hsub2((x & 0x00F000F0u) | magic, bias1);
+                    hi[2 * mi] = hsub2((y & 0x000F000Fu) | magic, bias2);
+                    hi[2 * mi + 1] = hsub2((y & 0x00F000F0u) | magic, bias3);
                 }
+                const uint32_t col = (uint32_t)(ts * 32 + 16 * hh);
+                ptx::tmem_st_16x128b_x4(lane_base + col, lo);
+                ptx::tmem_st_16x128b_x4(lane_base + (16u << 16) + col, hi);
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_addr(&bar_afull[ts]));
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ----------------------------------------------------------- MMA issuer
         // The whole warp runs the loop (so the operands stay warp-uniform) and one elected lane
-        // issues the MMAs and commits: measured on B200, issuing from a lane-0-only branch cost
-        // about 240 cycles per tcgen05.mma.
+        // issues the MMAs and commits.
         const bool leader = ptx::elect_one();
         const uint32_t idesc = idesc_f16<MN>();
         int sg = 0;              // segment counter
-        uint32_t acc = 0;
-        // Segments of 16-k steps end at a group boundary or at the slab end; tracked incrementally.
-        int64_t seg_next = (seg.k_lo / p.G + 1) * p.G;   // next group boundary after the slab start
-        bool starts = true;
-        for (int i = 0; i < nst; ++i) {
-            const int s = i % SS, ts = i % kTmemStages;
-            bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort, p.wait_ns);
-            okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns);
-            if (!__all_sync(0xffffffffu, okw)) break;
-            ptx::tc_fence_after();
-            const uint32_t bbase = ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes);
+        if constexpr (FAST) {
+            // Segments are whole stages: `rem` counts the stages left in the open group. The stage
+            // loop is unrolled over the ring, so slot, A-slot and B-descriptor offsets are constants.
+            const int gs = p.G / kStageK;
+            int rem = gs - (int)(st_lo % gs);
+            const uint64_t bdesc0 = kmajor_sw128_desc(ptx::smem_addr(s_b));
+            const uint32_t t_d = tmem + (uint32_t)C::kDCol;
             bool ok = true;
+            for (int i0 = 0; i0 < nst && ok; i0 += SS) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int64_t k = (st_lo + i) * kStageK + 16 * j;
-                const int db = sg & 1;
-                const bool ends = k + 16 == seg.k_hi || k + 16 == seg_next;
-                if (k + 16 == seg_next) seg_next += p.G;
-                if (starts) {
-                    const bool okd = ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1, &s_abort,
+                for (int u = 0; u < SS; ++u) {
+                    const int i = i0 + u;
+                    if (i >= nst) break;
+                    constexpr int kTsMask = kTmemStages - 1;
+                    const int ts = u & kTsMask;
+                    const bool seg_start = rem == gs || i == 0;
+                    const bool seg_end = rem == 1 || i == nst - 1;
+                    const int db = sg & 1;
+                    // The stage's A slot is complete only after every thread of its dequantiser group
+                    // has waited for the stage's TMA barrier, so this wait also orders the activation
+                    // tile before the MMAs (a second wait on that barrier cost ~150 cycles per stage).
+                    bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort,
+                                              p.wait_ns);
+                    if (seg_start)
+                        okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1, &s_abort,
                                                     p.wait_ns);
-                    if (!__all_sync(0xffffffffu, okd)) {
+                    if (!__all_sync(0xffffffffu, okw)) {
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after();
-                    acc = 0;
-                }
-                if (leader)
-                    ptx::mma_f16_ts(tmem + (uint32_t)(C::kDCol + db * MN), tmem + (uint32_t)(ts * 32 + 8 * j),
-                                    kmajor_sw128_desc(bbase + 32 * j), idesc, acc);
-                acc = 1;
-                starts = ends;
-                if (ends) {
-                    if (leader) ptx::mma_commit(ptx::smem_addr(&bar_dfull[db]));
-                    ++sg;
+                    if (leader) {
+                        const uint32_t d = t_d + (uint32_t)(db * MN);
+                        const uint32_t a = tmem + (uint32_t)(ts * 32);
+                        const uint64_t b = bdesc0 + (uint64_t)((u * C::kBStageBytes) >> 4);
+                        ptx::mma_f16_ts(d, a, b, idesc, seg_start ? 0u : 1u);
+                        ptx::mma_f16_ts(d, a + 8, b + 2, idesc, 1u);     // +32 B of B: 2 descriptor units
+                        ptx::mma_f16_ts(d, a + 16, b + 4, idesc, 1u);
+                        ptx::mma_f16_ts(d, a + 24, b + 6, idesc, 1u);
+                        if (seg_end) ptx::mma_commit(ptx::smem_addr(&bar_dfull[db]));
+                        ptx::mma_commit(ptx::smem_addr(&bar_empty[u]));
+                        ptx::mma_commit(ptx::smem_addr(&bar_aempty[ts]));
+                    }
+                    __syncwarp();
+                    if (seg_end) {
+                        ++sg;
+                        rem = gs;
+                    } else {
+                        --rem;
+                    }
                 }
             }
-            if (leader) {
-                ptx::mma_commit(ptx::smem_addr(&bar_empty[s]));
-                ptx::mma_commit(ptx::smem_addr(&bar_aempty[ts]));
+        } else {
+            uint32_t acc = 0;
+            // Segments of 16-k steps end at a group boundary or at the slab end; tracked incrementally.
+            int64_t seg_next = (seg.k_lo / p.G + 1) * p.G;   // next group boundary after the slab start
+            bool starts = true;
+            for (int i = 0; i < nst; ++i) {
+                const int s = i % SS, ts = i % kTmemStages;
+                bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort, p.wait_ns);
+                okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns);
+                if (!__all_sync(0xffffffffu, okw)) break;
+                ptx::tc_fence_after();
+                const uint32_t bbase = ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes);
+                bool ok = true;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t k = (st_lo + i) * kStageK + 16 * j;
+                    const int db = sg & 1;
+                    const bool ends = k + 16 == seg.k_hi || k + 16 == seg_next;
+                    if (k + 16 == seg_next) seg_next += p.G;
+                    if (starts) {
+                        const bool okd = ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1,
+                                                        &s_abort, p.wait_ns);
+                        if (!__all_sync(0xffffffffu, okd)) {
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        acc = 0;
+                    }
+                    if (leader)
+                        ptx::mma_f16_ts(tmem + (uint32_t)(C::kDCol + db * MN), tmem + (uint32_t)(ts * 32 + 8 * j),
+                                        kmajor_sw128_desc(bbase + 32 * j), idesc, acc);
+                    acc = 1;
+                    starts = ends;
+                    if (ends) {
+                        if (leader) ptx::mma_commit(ptx::smem_addr(&bar_dfull[db]));
+                        ++sg;
+                    }
+                }
+                if (leader) {
+                    ptx::mma_commit(ptx::smem_addr(&bar_empty[s]));
+                    ptx::mma_commit(ptx::smem_addr(&bar_aempty[ts]));
+                }
+                __syncwarp();
+                if (!ok) break;
             }
-            __syncwarp();
-            if (!ok) break;
         }
         // Wait for every MMA issued above before TMEM can be released.
         if (leader) ptx::mma_commit(ptx::smem_addr(&bar_drain));
@@ -312,7 +392,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     } else {
         // -------------------------------------------------------------- epilogue
         const int sub = warp & 3;                           // TMEM lanes 32 sub .. 32 sub + 31
-        const int et = threadIdx.x - 192;                   // 0..127 within the epilogue warps
+        const int et = threadIdx.x - 32 * kEpiWarp0;        // 0..127 within the epilogue warps
         const int ncol = 32 * sub + 4 * (lane & 7) + (lane >> 3);
         const int64_t n = (int64_t)tile * kBlockN + ncol;
         const float fscale = (lane >> 3) & 1 ? 0.0625f : 1.0f;
@@ -390,7 +470,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     ptx::tc_fence_before();
     __syncthreads();
     if (s_abort && threadIdx.x == 0 && p.status) atomicExch(p.status, (int)W4A16_ERR_TIMEOUT);
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, C::kTmemCols);
     }
@@ -398,18 +478,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 
 using TcFn = void (*)(CUtensorMap, CUtensorMap, TcArgs);
 
-TcFn select_tc(int mn) {
+template <bool FAST>
+TcFn select_tc_t(int mn) {
     switch (mn) {
-        case 16: return tc_gemm_kernel<16>;
-        case 32: return tc_gemm_kernel<32>;
-        case 48: return tc_gemm_kernel<48>;
-        case 64: return tc_gemm_kernel<64>;
-        case 80: return tc_gemm_kernel<80>;
-        case 96: return tc_gemm_kernel<96>;
-        case 112: return tc_gemm_kernel<112>;
-        default: return tc_gemm_kernel<128>;
+        case 16: return tc_gemm_kernel<16, FAST>;
+        case 32: return tc_gemm_kernel<32, FAST>;
+        case 48: return tc_gemm_kernel<48, FAST>;
+        case 64: return tc_gemm_kernel<64, FAST>;
+        case 80: return tc_gemm_kernel<80, FAST>;
+        case 96: return tc_gemm_kernel<96, FAST>;
+        case 112: return tc_gemm_kernel<112, FAST>;
+        default: return tc_gemm_kernel<128, FAST>;
     }
 }
+TcFn select_tc(int mn, bool fast) { return fast ? select_tc_t<true>(mn) : select_tc_t<false>(mn); }
 
 size_t tc_smem(int mn) {
     switch (mn) {
@@ -432,14 +514,14 @@ int tc_ctas_per_sm(int mn) {
     // Resident CTAs per SM from the three budgets the kernel draws on: shared
     // memory (228 KB per SM, 1 KB reserved per CTA), registers (64 K per SM)
     // and tensor memory (512 columns per SM).
-    TcFn k = select_tc(mn);
+    TcFn k = select_tc(mn, true);
     const size_t smem = tc_smem(mn);
     cudaFuncAttributes fa{};
     int regs = 255;
     if (cudaFuncGetAttributes(&fa, k) == cudaSuccess && fa.numRegs > 0) regs = fa.numRegs;
     const int by_smem = (int)((228 * 1024) / (smem + fa.sharedSizeBytes + 1024));
     const int regs_per_warp = (regs + 7) / 8 * 8 * 32;  // allocation granularity: 8 registers per thread
-    const int by_regs = 65536 / (regs_per_warp * (kThreadsTC / 32));
+    const int by_regs = 65536 / (regs_per_warp * (tc_threads(mn) / 32));
     const int cols = mn <= 64 ? 256 : 512;
     n = std::max(1, std::min(std::min(by_smem, by_regs), 512 / cols));
     g_tc_occ[mn / 16].store(n, std::memory_order_relaxed);
@@ -528,11 +610,11 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
         args.wait_ns = wp.limit_ns;
         // Every row block uses the plan's MN (the largest); a short last block
         // leaves its padded rows to TMA's zero fill.
-        TcFn k = select_tc(pl.mn);
+        TcFn k = select_tc(pl.mn, G % kStageK == 0);
         const size_t smem = tc_smem(pl.mn);
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        k<<<dim3((unsigned)pl.n_tiles, (unsigned)pl.split_k), kThreadsTC, smem, st>>>(amap, wmap, args);
+        k<<<dim3((unsigned)pl.n_tiles, (unsigned)pl.split_k), tc_threads(pl.mn), smem, st>>>(amap, wmap, args);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
