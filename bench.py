@@ -172,12 +172,19 @@ class Problem:
                           workspace=self.ws, stream=stream, pdl=self.pdl)
 
     def launches_per_step(self):
-        # GEMV (one launch per 16 rows) for M <= 32; tensor-core GEMM (one per 128 rows) above.
-        return (self.M + 15) // 16 if self.M <= 32 else (self.M + 127) // 128
+        # The library's automatic choice: tensor-core GEMM (one launch per 128 rows) above 32 rows,
+        # and for 17..32 rows when N has at least 96 tiles of 128 columns; otherwise the GEMV (one
+        # launch per 16 rows).
+        return (self.M + 127) // 128 if uses_tc(self.M, self.N) else (self.M + 15) // 16
 
 
 def copies_for(bytes_per_copy):
     return max(2, int(np.ceil(2 * L2_BYTES / bytes_per_copy)) + 1)
+
+
+def uses_tc(M, N):
+    """The library's automatic kernel choice for an aligned problem (see w4a16_api.cu)."""
+    return M > 32 or (M > 16 and N // 128 >= 96)
 
 
 def capture(torch, fn, n):
@@ -337,8 +344,8 @@ def run_gpu(args):
     Problem.pdl = args.pdl
     achieved = prob.bytes / per_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
-    kernel_name = "gemv_sk_kernel<16, true>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
-    traffic = traffic_from_profiles("gemv_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
+    kernel_name = "tc_gemm_kernel<32, true>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
+    traffic = traffic_from_profiles("tc_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
     if traffic is not None:  # per step, like `achieved` (the batch-32 step is two 16-row launches)
         traffic = traffic * prob.launches_per_step()
 

@@ -125,7 +125,7 @@ struct SegIter {
 
 // FAST: G is a multiple of the 64-row stage, so group segments are whole stages.
 template <int MN, bool FAST>
-__global__ void __launch_bounds__(tc_threads(MN), (TcCfg<MN>::kTmemCols <= 256 && MN <= 32) ? 2 : 1)
+__global__ void __launch_bounds__(tc_threads(MN), 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap, TcArgs p) {
     using C = TcCfg<MN>;
     constexpr int kDeqWarps = deq_warps(MN);
@@ -224,6 +224,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         uint32_t bias0 = 0, bias1 = 0, bias2 = 0, bias3 = 0;
         const uint32_t magic = p.magic;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        // (1024 + z) for low-nibble columns, (1024 + 16 z) for high ones, in both halves
+        auto set_bias = [&](uint32_t zw) {
+            bias0 = (0x6400u + (zw & 0xFu)) * 0x00010001u;
+            bias1 = (0x6400u + 16u * ((zw >> 4) & 0xFu)) * 0x00010001u;
+            bias2 = (0x6400u + ((zw >> 8) & 0xFu)) * 0x00010001u;
+            bias3 = (0x6400u + 16u * ((zw >> 12) & 0xFu)) * 0x00010001u;
+        };
         auto enter_group = [&](int64_t kk) {
             const int64_t g = kk / p.G;
             g_next_k = (g + 1) * p.G;
@@ -234,13 +241,24 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 have_next = g_pref < ngroups;
                 if (have_next) zw_next = __ldg(p.z + g_pref * nw + word);
             }
-            const uint32_t zw = p.z ? (zraw >> (4 * nib0)) : (uint32_t)p.zp_bias * 0x1111u;
-            // (1024 + z) for low-nibble columns, (1024 + 16 z) for high ones, in both halves
-            bias0 = (0x6400u + (zw & 0xFu)) * 0x00010001u;
-            bias1 = (0x6400u + 16u * ((zw >> 4) & 0xFu)) * 0x00010001u;
-            bias2 = (0x6400u + ((zw >> 8) & 0xFu)) * 0x00010001u;
-            bias3 = (0x6400u + 16u * ((zw >> 12) & 0xFu)) * 0x00010001u;
+            set_bias(p.z ? (zraw >> (4 * nib0)) : (uint32_t)p.zp_bias * 0x1111u);
         };
+        // FAST: one group per stage; the zero words of my next four stages are loaded ahead in a
+        // register ring (a DRAM round trip is longer than one or two stages).
+        auto zero_of_stage = [&](int st) -> uint32_t {
+            return (p.z && st < nst) ? __ldg(p.z + (st_lo + st) * kStageK / p.G * nw + word) : 0u;
+        };
+        uint32_t zr0 = 0u, zr1 = 0u, zr2 = 0u, zr3 = 0u;
+        if (FAST) {
+            if (p.z) {
+                zr0 = zero_of_stage(dg);
+                zr1 = zero_of_stage(dg + kDeqGroups);
+                zr2 = zero_of_stage(dg + 2 * kDeqGroups);
+                zr3 = zero_of_stage(dg + 3 * kDeqGroups);
+            } else {
+                set_bias((uint32_t)p.zp_bias * 0x1111u);
+            }
+        }
         for (int i = dg; i < nst; i += kDeqGroups) {
             const int s = i % SS, ts = i % kTmemStages;
             // Wait outcomes are made warp-uniform: the tcgen05 stores below are .sync.aligned.
@@ -250,6 +268,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             if (!__all_sync(0xffffffffu, okw)) break;
             ptx::tc_fence_after();
             const uint32_t wbase = ptx::smem_addr(s_w + (size_t)s * kWStageBytes);
+            if (FAST && p.z) {
+                set_bias(zr0 >> (4 * nib0));
+                zr0 = zr1;
+                zr1 = zr2;
+                zr2 = zr3;
+                zr3 = zero_of_stage(i + 4 * kDeqGroups);
+            }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 // rows 32hh .. 32hh + 31 as four 8x8 matrices of 16-bit halves; my address row is
@@ -258,7 +283,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 uint32_t R[4];
                 ptx::ldmatrix_x4_trans(wbase + row * 64 + 16 * (q ^ ((row >> 1) & 3)), R);
                 const int64_t k_half = (st_lo + i) * kStageK + 32 * hh;   // first k of this half stage
-                if (FAST && k_half >= g_next_k) enter_group(k_half);       // groups start at stage starts only
                 uint32_t lo[8], hi[8];
 #pragma unroll
                 for (int mi = 0; mi < 4; ++mi) {
@@ -401,16 +425,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         for (int m = 0; m < MN; ++m) tot[m] = 0.f;
         int sg = 0;
         bool ok = true;
-        // Segment ends in order (group boundaries, tracked incrementally); each segment's scale is
-        // loaded one segment ahead.
+        // Segment ends in order (group boundaries, tracked incrementally).
         int64_t g_idx = seg.k_lo / p.G;                    // group of the current segment
         int64_t bound = (g_idx + 1) * p.G;                 // its end row (or the slab end)
-        auto scale_of = [&](int64_t g) -> float { return fscale * __half2float(p.s[g * p.N + n]); };
+        const int64_t g_last = (seg.k_hi - 1) / p.G;       // last group of the slab
+        // Segments are consecutive groups; their scales are loaded four segments ahead in a
+        // register ring (a DRAM round trip is longer than one segment).
+        auto scale_of = [&](int64_t g) -> float {
+            return g <= g_last ? fscale * __half2float(p.s[g * p.N + n]) : 0.f;
+        };
         int64_t k_end = min(seg.k_hi, bound) - 16;
-        float sc = scale_of(g_idx);
+        float sc = scale_of(g_idx), sc1 = scale_of(g_idx + 1), sc2 = scale_of(g_idx + 2), sc3 = scale_of(g_idx + 3);
         while (k_end >= seg.k_lo && ok) {
             const int64_t k_next = k_end + 16 < seg.k_hi ? min(seg.k_hi, bound + p.G) - 16 : -1;
-            const float sc_next = k_next >= 0 ? scale_of(g_idx + 1) : 0.f;
+            const float sc_next = sc1;
+            sc1 = sc2;
+            sc2 = sc3;
+            sc3 = scale_of(g_idx + 4);
             const int db = sg & 1;
             const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_dfull[db]), (sg >> 1) & 1, &s_abort, p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) {  // warp-uniform: tcgen05.ld is .sync.aligned
@@ -506,6 +537,12 @@ size_t tc_smem(int mn) {
     }
 }
 
+// Dynamic shared memory requested at launch. Shapes up to 32 rows ask for more than half of an
+// SM's 228 KB so that each CTA has an SM to itself: measured on B200 (K=4096, N=14336, M=32),
+// two CTAs per SM with the K range split in two ran 41.5 us against 31.8 us for 48 rows with one
+// CTA per SM and no split.
+size_t tc_launch_smem(int mn) { return mn <= 32 ? std::max<size_t>(tc_smem(mn), 116 * 1024) : tc_smem(mn); }
+
 std::atomic<int> g_tc_occ[9];
 
 int tc_ctas_per_sm(int mn) {
@@ -515,7 +552,7 @@ int tc_ctas_per_sm(int mn) {
     // memory (228 KB per SM, 1 KB reserved per CTA), registers (64 K per SM)
     // and tensor memory (512 columns per SM).
     TcFn k = select_tc(mn, true);
-    const size_t smem = tc_smem(mn);
+    const size_t smem = tc_launch_smem(mn);
     cudaFuncAttributes fa{};
     int regs = 255;
     if (cudaFuncGetAttributes(&fa, k) == cudaSuccess && fa.numRegs > 0) regs = fa.numRegs;
@@ -611,7 +648,7 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
         // Every row block uses the plan's MN (the largest); a short last block
         // leaves its padded rows to TMA's zero fill.
         TcFn k = select_tc(pl.mn, G % kStageK == 0);
-        const size_t smem = tc_smem(pl.mn);
+        const size_t smem = tc_launch_smem(pl.mn);
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         k<<<dim3((unsigned)pl.n_tiles, (unsigned)pl.split_k), tc_threads(pl.mn), smem, st>>>(amap, wmap, args);

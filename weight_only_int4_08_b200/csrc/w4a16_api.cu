@@ -81,13 +81,20 @@ struct Choice {
     TcPlan tc;
 };
 
-// Kernel table: the mma.sync GEMV for M <= 32 (one launch per 16 rows; the
-// CUDA-core GEMV when its alignment rules fail), the tensor-core GEMM above when
-// the shape and pointers allow it (N % 128, K % 64, 16-byte aligned A and
-// weights), the GEMV's row blocks otherwise. Null pointers (workspace query)
-// count as aligned. Measured on B200 (K=4096, N=14336, M=32): two 16-row GEMV
-// launches 35.6 us, the tensor-core GEMM 41.4 us (28.6 us at M=64).
-constexpr int64_t kGemvMaxM = 32;
+// Kernel table. M <= 16: the mma.sync GEMV (one launch; the CUDA-core GEMV when its
+// alignment rules fail). 17..32 rows: the GEMV needs two launches, each reading all the
+// weights, while the tensor-core GEMM reads them once, one CTA per 128 columns; the GEMM is
+// taken when N has at least 96 such column tiles. Above 32 rows: the GEMM. The GEMM only
+// when the shape and pointers allow it (N % 128, K % 64, 16-byte aligned A and weights),
+// the GEMV's row blocks otherwise. Null pointers (workspace query) count as aligned.
+// Measured on B200 at M=32, G=128, CUDA graphs, weights larger than L2 (GEMV / GEMM):
+// K=4096 N=14336 37.6 / 31.2 us; N=28672 72.8 / 49.2 us; N=6144 31.6 / 35.0 us;
+// N=4096 25.5 / 27.5 us; K=14336 N=4096 41.3 / 40.3 us. At K=4096 N=14336 the GEMM is
+// ahead from 17 rows (31.2 / 30.3 us).
+constexpr int64_t kGemvOneLaunchM = 16, kGemvMaxM = 32, kTcMinTiles = 96;
+bool auto_prefers_tc(int64_t M, int64_t N) {
+    return M > kGemvMaxM || (M > kGemvOneLaunchM && N / 128 >= kTcMinTiles);
+}
 Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms,
               const void* a, const void* b, const void* s) {
     Choice c{};
@@ -95,7 +102,7 @@ Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_optio
     const bool tc_ok = tc_supported(M, N, K, G, a ? a : (const void*)16, b ? b : (const void*)16);
     if (req == W4A16_KERNEL_TC) c.kernel = W4A16_KERNEL_TC;
     else if (req == W4A16_KERNEL_GEMV || req == W4A16_KERNEL_GEMV_FMA) c.kernel = W4A16_KERNEL_GEMV;
-    else c.kernel = (M > kGemvMaxM && tc_ok) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
+    else c.kernel = (auto_prefers_tc(M, N) && tc_ok) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
     const int split = opts ? opts->split_k : 0;
     if (c.kernel == W4A16_KERNEL_TC) {
         if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, split);
@@ -120,7 +127,7 @@ size_t ws_bound(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_opt
         if (req != W4A16_KERNEL_GEMV_FMA && N % 32 == 0) ws = std::max(ws, plan_gemv_mma(M, N, K, G, split, sms).ws_bytes);
     }
     const bool tc_shape = tc_supported(M, N, K, G, (const void*)16, (const void*)16);
-    if (tc_shape && (req == W4A16_KERNEL_TC || (req == W4A16_KERNEL_AUTO && M > kGemvMaxM)))
+    if (tc_shape && (req == W4A16_KERNEL_TC || (req == W4A16_KERNEL_AUTO && auto_prefers_tc(M, N))))
         ws = std::max(ws, plan_tc(M, N, K, G, sms, opts ? opts->split_k : 0).ws_bytes);
     return ws;
 }
