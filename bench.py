@@ -66,22 +66,24 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def csrc_hash():
+def csrc_hash(files=None):
+    """Hash of the library sources a kernel is compiled from (all of csrc/ when files is None)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "weight_only_int4_08_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files or os.listdir(d)):
         h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def traffic_from_profiles(kernel_key):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+    """DRAM bytes per launch from the committed ncu summary, if the sources of that kernel (its
+    translation unit and the headers it includes) are the ones it was taken on."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(kernel_key)
-    if not e or e.get("csrc_hash") != csrc_hash():
+    if not e or e.get("csrc_hash") != csrc_hash(e.get("files")):
         return None
     return e.get("dram_bytes_per_launch")
 
