@@ -234,6 +234,21 @@ def summary(prob, per_step_s, peaks, tensor_bound):
             "roofline_us": round(t_roof * 1e6, 3), "frac_of_roofline": round(t_roof / per_step_s, 4)}
 
 
+def max_over_ranks(dist, world, seconds, device):
+    """The job's time: the largest of the ranks' local times, returned on every rank."""
+    if world <= 1:
+        return seconds
+    import torch
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world, steps, bytes_per_step, seconds):
+    """Whole-job throughput: each of the `world` ranks ran `steps` steps of `bytes_per_step`."""
+    return world * steps * bytes_per_step / seconds / 1e9
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -298,13 +313,9 @@ def run_gpu(args):
         torch.cuda.synchronize()
     clocks = sampler.stop()
 
-    t_max = t_local
-    if world > 1:
-        tt = torch.tensor([t_local], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
+    t_max = max_over_ranks(dist, world, t_local, "cuda")
     per_step = t_max / K_steps
-    value = world * K_steps * prob.bytes / t_max / 1e9
+    value = whole_job_gbs(world, K_steps, prob.bytes, t_max)
 
     # e2e: through the public API with pinned host buffers; H2D of the step's
     # activations and D2H of its output inside the timed region, every step.
@@ -331,12 +342,8 @@ def run_gpu(args):
     f1.record()
     torch.cuda.synchronize()
     barrier()
-    te = f0.elapsed_time(f1) / 1e3
-    if world > 1:
-        tt = torch.tensor([te], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        te = float(tt.item())
-    e2e_value = world * e2e_steps * prob.bytes / te / 1e9
+    te = max_over_ranks(dist, world, f0.elapsed_time(f1) / 1e3, "cuda")
+    e2e_value = whole_job_gbs(world, e2e_steps, prob.bytes, te)
 
     # kernel duration for the roofline: graph of back-to-back launches, CUDA events
     per_launch = measure_problem(torch, prob, 256, 40)
@@ -348,7 +355,7 @@ def run_gpu(args):
     hbm_peak = float(peaks["hbm_gbs"])
     kernel_name = "tc_gemm_kernel<32, true>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
     traffic = traffic_from_profiles("tc_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
-    if traffic is not None:  # per step, like `achieved` (the batch-32 step is two 16-row launches)
+    if traffic is not None:  # per step, like `achieved`
         traffic = traffic * prob.launches_per_step()
 
     extras = {}
