@@ -63,22 +63,26 @@ __device__ __forceinline__ void repack_tile(const uint32_t* __restrict__ ckpt, u
     const int64_t n0 = by * kTileRows;    // first n row
 
     const int64_t kw = kw0 + lane;
-    // Each warp transposes n-blocks b = warp, warp + 8, warp + 16, warp + 24.
+    // Each warp transposes n-blocks b = warp, warp + 8, warp + 16, warp + 24. All 32 loads are
+    // issued before the first transpose, so that each thread keeps 128 bytes in flight.
+    constexpr int kBlocks = kTileWords / 8;
+    uint32_t x[kBlocks][8];
 #pragma unroll
-    for (int bb = 0; bb < kTileWords / 8; ++bb) {
-        const int b = warp + 8 * bb;
-        uint32_t x[8];
+    for (int bb = 0; bb < kBlocks; ++bb)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int64_t n = n0 + 8 * b + i;
-            x[i] = (n < N && kw < kw_total) ? __ldg(ckpt + n * kw_total + kw) : 0u;
+            const int64_t n = n0 + 8 * (warp + 8 * bb) + i;
+            x[bb][i] = (n < N && kw < kw_total) ? __ldg(ckpt + n * kw_total + kw) : 0u;
         }
-        nibble_transpose8(x);
-        // x[i] now holds q[k = 8*kw + i, n = n0 + 8b .. n0 + 8b + 7]
+#pragma unroll
+    for (int bb = 0; bb < kBlocks; ++bb) {
+        const int b = warp + 8 * bb;
+        nibble_transpose8(x[bb]);
+        // x[bb][i] now holds q[k = 8*kw + i, n = n0 + 8b .. n0 + 8b + 7]
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int r = 8 * lane + i;  // k_local; r / 8 == lane
-            tile[r * kTileWords + (b ^ lane)] = x[i];
+            tile[r * kTileWords + (b ^ lane)] = x[bb][i];
         }
     }
     __syncthreads();
