@@ -159,7 +159,7 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  * Kernel selection for tests and measurement.
  *   kernel: W4A16_KERNEL_AUTO uses the same table as w4a16_gemm (GEMV for
  *     M <= 16, and for 17..32 rows when N / 128 < 96; tensor cores otherwise
- *     when N % 128 == 0, K % 64 == 0 and a, b_packed are 16-byte aligned); GEMV forces the GEMV family (any M; larger
+ *     when N % 128 == 0, K % 128 == 0 and a, b_packed are 16-byte aligned); GEMV forces the GEMV family (any M; larger
  *     M runs it once per block of 16 rows of A): its multiply-accumulate uses
  *     warp mma.sync when N % 32 == 0, a and b_packed are 16-byte and scales
  *     8-byte aligned, the CUDA-core fp32 loop (8-row blocks) otherwise;

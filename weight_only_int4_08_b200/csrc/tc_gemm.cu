@@ -14,10 +14,11 @@
 //
 // Roles (one CTA = one 128-column tile x one K slab; 14 warps, 10 above MN = 64;
 // the warp numbers below are those of the 14-warp form):
-//   warp 8      producer: per stage of 64 k-rows, one 2-D TMA load of the
-//               tile's packed words [64 rows x 64 B] (64-byte swizzle) and one of
+//   warp 8      producer: per stage of 128 k-rows, one 2-D TMA load of the
+//               tile's packed words [128 rows x 64 B] (64-byte swizzle) and two of
 //               the activation tile [MN x 64] (128-byte swizzle, the canonical
-//               K-major layout of operand B), into an 8-stage ring;
+//               K-major layout of operand B), into an 8-stage ring (4 above
+//               MN = 64);
 //   warps 0-7   dequantisers (0-3 above MN = 64): warp p owns TMEM lanes
 //               32(p%4)..+31 and tile columns 32(p%4)..+31 (one 16-byte chunk of
 //               each weight row); warps 0-3 take the even stages and 4-7 the odd
@@ -25,10 +26,10 @@
 //               per register, which become exact fp16 (q - z) pairs (0x6400 magic
 //               + fp16 subtract) written to TMEM with tcgen05.st.16x128b.x4;
 //   warp 9      TMEM allocator and MMA issuer: tcgen05.mma.kind::f16 with A
-//               from TMEM and B from shared memory, 4 per stage (K = 16 each);
+//               from TMEM and B from shared memory, 8 per stage (K = 16 each);
 //               a fresh accumulator per group segment, double-buffered, and a
 //               tcgen05.commit to an mbarrier at each segment end. When G is a
-//               multiple of 64 (segments are whole stages) the stage loop is
+//               multiple of 128 (segments are whole stages) the stage loop is
 //               unrolled over the ring so that every operand address is a
 //               constant offset: measured on B200, the issue loop's own
 //               instructions and barrier waits, not the tensor core, set the
@@ -59,9 +60,13 @@ namespace {
 
 constexpr int kBlockN = 128;                    // MMA M = TMEM lanes = output columns per CTA
 constexpr int kTileWords = kBlockN / 8;         // 16 packed words per k-row of the tile
-constexpr int kStageK = 64;                     // k-rows per pipeline stage
-constexpr int kWStageBytes = kStageK * kTileWords * 4;   // 64 rows x 64 B, 64-byte swizzle
-constexpr int kTmemStages = 4;                  // A slots in TMEM (32 columns = 64 k each)
+constexpr int kStageK = 128;                    // k-rows per pipeline stage
+constexpr int kWStageBytes = kStageK * kTileWords * 4;   // 128 rows x 64 B, 64-byte swizzle
+constexpr int kBoxK = 64;                       // activation TMA box width (128 B: the 128-byte swizzle's limit)
+constexpr int kBoxes = kStageK / kBoxK;         // activation boxes per stage
+constexpr int kMmaPerStage = kStageK / 16;      // K = 16 per tcgen05.mma.kind::f16
+constexpr int kAColsPerStage = kStageK / 2;     // TMEM columns of one A slot (two fp16 per column)
+constexpr int kTmemStages = 4;                  // A slots in TMEM
 // Dequantiser warps: groups of four (one per TMEM lane quarter) that take turns on the stages,
 // two groups while the MMAs are short (MN <= 64), one above, where the per-column totals of
 // the epilogue need the registers that more threads would take. A group's stage ends with a
@@ -71,9 +76,11 @@ __host__ __device__ constexpr int tc_threads(int mn) { return (deq_warps(mn) + 6
 
 template <int MN>
 struct TcCfg {
-    static constexpr int kSmemStages = 8;   // a multiple of kTmemStages (the unrolled issue loop relies on it)
-    static constexpr int kBStageBytes = MN * 128;           // MN rows x 64 k x 2 B
-    static constexpr int kDCol = kTmemStages * 32;          // first accumulator column
+    // a multiple of kTmemStages (the unrolled issue loop relies on it)
+    static constexpr int kSmemStages = MN <= 64 ? 8 : 4;
+    static constexpr int kBoxBytes = MN * kBoxK * 2;        // one activation box: MN rows x 128 B
+    static constexpr int kBStageBytes = kBoxes * kBoxBytes;
+    static constexpr int kDCol = kTmemStages * kAColsPerStage;   // first accumulator column
     static constexpr int kColsNeeded = kDCol + 2 * MN;
     static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64 : kColsNeeded <= 128 ? 128
                                    : kColsNeeded <= 256 ? 256 : 512;
@@ -123,7 +130,7 @@ struct SegIter {
     int G;
 };
 
-// FAST: G is a multiple of the 64-row stage, so group segments are whole stages.
+// FAST: G is a multiple of the stage (kStageK rows), so group segments are whole stages.
 template <int MN, bool FAST>
 __global__ void __launch_bounds__(tc_threads(MN), 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap, TcArgs p) {
@@ -134,8 +141,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     extern __shared__ __align__(1024) unsigned char s_raw[];
     unsigned char* s_base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(s_raw) + 1023) & ~(uintptr_t)1023);
-    unsigned char* s_b = s_base;                                   // [SS][MN x 128 B], 1024-aligned stages
-    unsigned char* s_w = s_base + (size_t)SS * C::kBStageBytes;    // [SS][64 rows x 64 B], 1024-aligned stages
+    unsigned char* s_b = s_base;                                   // [SS][2][MN x 128 B], 1024-aligned boxes
+    unsigned char* s_w = s_base + (size_t)SS * C::kBStageBytes;    // [SS][128 rows x 64 B], 1024-aligned stages
 
     __shared__ __align__(8) uint64_t bar_full[SS], bar_empty[SS];
     __shared__ __align__(8) uint64_t bar_afull[kTmemStages], bar_aempty[kTmemStages];
@@ -196,7 +203,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 ptx::mbar_arrive_expect_tx(full, tx);
                 const int32_t k0 = (int32_t)((st_lo + i) * kStageK);
                 ptx::tma_load_2d(ptx::smem_addr(s_w + (size_t)s * kWStageBytes), &wmap, tile * kTileWords, k0, full);
-                ptx::tma_load_2d(ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes), &amap, k0, p.m0, full);
+#pragma unroll
+                for (int x = 0; x < kBoxes; ++x)
+                    ptx::tma_load_2d(ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes + x * C::kBoxBytes), &amap,
+                                     k0 + x * kBoxK, p.m0, full);
             }
             __syncwarp();
             issued = i + 1;
@@ -276,13 +286,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 zr3 = zero_of_stage(i + 4 * kDeqGroups);
             }
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
+            for (int hh = 0; hh < kStageK / 32; ++hh) {
                 // rows 32hh .. 32hh + 31 as four 8x8 matrices of 16-bit halves; my address row is
                 // 32hh + lane; 16-byte chunk q of it, moved by the 64-byte swizzle
                 const int row = 32 * hh + lane;
                 uint32_t R[4];
                 ptx::ldmatrix_x4_trans(wbase + row * 64 + 16 * (q ^ ((row >> 1) & 3)), R);
-                const int64_t k_half = (st_lo + i) * kStageK + 32 * hh;   // first k of this half stage
+                const int64_t k_half = (st_lo + i) * kStageK + 32 * hh;   // first k of these 32 rows
                 uint32_t lo[8], hi[8];
 #pragma unroll
                 for (int mi = 0; mi < 4; ++mi) {
@@ -294,7 +304,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     hi[2 * mi] = hsub2((y & 0x000F000Fu) | magic, bias2);
                     hi[2 * mi + 1] = hsub2((y & 0x00F000F0u) | magic, bias3);
                 }
-                const uint32_t col = (uint32_t)(ts * 32 + 16 * hh);
+                const uint32_t col = (uint32_t)(ts * kAColsPerStage + 16 * hh);
                 ptx::tmem_st_16x128b_x4(lane_base + col, lo);
                 ptx::tmem_st_16x128b_x4(lane_base + (16u << 16) + col, hi);
             }
@@ -342,12 +352,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     ptx::tc_fence_after();
                     if (leader) {
                         const uint32_t d = t_d + (uint32_t)(db * MN);
-                        const uint32_t a = tmem + (uint32_t)(ts * 32);
+                        const uint32_t a = tmem + (uint32_t)(ts * kAColsPerStage);
                         const uint64_t b = bdesc0 + (uint64_t)((u * C::kBStageBytes) >> 4);
-                        ptx::mma_f16_ts(d, a, b, idesc, seg_start ? 0u : 1u);
-                        ptx::mma_f16_ts(d, a + 8, b + 2, idesc, 1u);     // +32 B of B: 2 descriptor units
-                        ptx::mma_f16_ts(d, a + 16, b + 4, idesc, 1u);
-                        ptx::mma_f16_ts(d, a + 24, b + 6, idesc, 1u);
+#pragma unroll
+                        for (int j = 0; j < kMmaPerStage; ++j) {
+                            // A: 8 TMEM columns per 16 k; B: box j / 4, +32 B (2 descriptor units) per 16 k
+                            const uint64_t bj = b + (uint64_t)(((j / 4) * C::kBoxBytes + 32 * (j % 4)) >> 4);
+                            ptx::mma_f16_ts(d, a + 8 * j, bj, idesc, (j == 0 && seg_start) ? 0u : 1u);
+                        }
                         if (seg_end) ptx::mma_commit(ptx::smem_addr(&bar_dfull[db]));
                         ptx::mma_commit(ptx::smem_addr(&bar_empty[u]));
                         ptx::mma_commit(ptx::smem_addr(&bar_aempty[ts]));
@@ -375,7 +387,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 const uint32_t bbase = ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes);
                 bool ok = true;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < kMmaPerStage; ++j) {
                     const int64_t k = (st_lo + i) * kStageK + 16 * j;
                     const int db = sg & 1;
                     const bool ends = k + 16 == seg.k_hi || k + 16 == seg_next;
@@ -391,8 +403,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                         acc = 0;
                     }
                     if (leader)
-                        ptx::mma_f16_ts(tmem + (uint32_t)(C::kDCol + db * MN), tmem + (uint32_t)(ts * 32 + 8 * j),
-                                        kmajor_sw128_desc(bbase + 32 * j), idesc, acc);
+                        ptx::mma_f16_ts(tmem + (uint32_t)(C::kDCol + db * MN),
+                                        tmem + (uint32_t)(ts * kAColsPerStage + 8 * j),
+                                        kmajor_sw128_desc(bbase + (j / 4) * C::kBoxBytes + 32 * (j % 4)), idesc, acc);
                     acc = 1;
                     starts = ends;
                     if (ends) {
@@ -559,7 +572,7 @@ int tc_ctas_per_sm(int mn) {
     const int by_smem = (int)((228 * 1024) / (smem + fa.sharedSizeBytes + 1024));
     const int regs_per_warp = (regs + 7) / 8 * 8 * 32;  // allocation granularity: 8 registers per thread
     const int by_regs = 65536 / (regs_per_warp * (tc_threads(mn) / 32));
-    const int cols = mn <= 64 ? 256 : 512;
+    const int cols = kTmemStages * kAColsPerStage + 2 * mn <= 256 ? 256 : 512;
     n = std::max(1, std::min(std::min(by_smem, by_regs), 512 / cols));
     g_tc_occ[mn / 16].store(n, std::memory_order_relaxed);
     return n;
@@ -612,7 +625,7 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
     CUtensorMap amap;
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kStageK, (cuuint32_t)pl.mn};
+    const cuuint32_t box[2] = {(cuuint32_t)kBoxK, (cuuint32_t)pl.mn};
     const cuuint32_t estr[2] = {1, 1};
     cudaError_t e = encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)a, dims, strides, box, estr,
                                       CU_TENSOR_MAP_SWIZZLE_128B);

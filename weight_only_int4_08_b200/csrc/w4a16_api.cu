@@ -85,12 +85,12 @@ struct Choice {
 // alignment rules fail). 17..32 rows: the GEMV needs two launches, each reading all the
 // weights, while the tensor-core GEMM reads them once, one CTA per 128 columns; the GEMM is
 // taken when N has at least 96 such column tiles. Above 32 rows: the GEMM. The GEMM only
-// when the shape and pointers allow it (N % 128, K % 64, 16-byte aligned A and weights),
+// when the shape and pointers allow it (N % 128, K % 128, 16-byte aligned A and weights),
 // the GEMV's row blocks otherwise. Null pointers (workspace query) count as aligned.
 // Measured on B200 at M=32, G=128, CUDA graphs, weights larger than L2 (GEMV / GEMM):
-// K=4096 N=14336 37.6 / 31.2 us; N=28672 72.8 / 49.2 us; N=6144 31.6 / 35.0 us;
-// N=4096 25.5 / 27.5 us; K=14336 N=4096 41.3 / 40.3 us. At K=4096 N=14336 the GEMM is
-// ahead from 17 rows (31.2 / 30.3 us).
+// K=4096 N=14336 37.6 / 20.6 us; N=28672 72.7 / 41.2 us; N=6144 31.8 / 33.0 us;
+// N=4096 25.8 / 25.8 us; K=14336 N=4096 41.5 / 36.2 us. At K=4096 N=14336 the GEMM is
+// ahead from 17 rows (31.2 / 19.8 us).
 constexpr int64_t kGemvOneLaunchM = 16, kGemvMaxM = 32, kTcMinTiles = 96;
 bool auto_prefers_tc(int64_t M, int64_t N) {
     return M > kGemvMaxM || (M > kGemvOneLaunchM && N / 128 >= kTcMinTiles);
@@ -283,7 +283,7 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
     }
     Choice c = choose(M, N, K, group_size, opts, sms, a, b_packed, scales);
     if (c.kernel == W4A16_KERNEL_TC && !tc_supported(M, N, K, group_size, a, b_packed)) {
-        set_error("unsupported: %s", "tensor-core kernel needs N % 128 == 0, K % 64 == 0, 16-byte aligned a and b_packed");
+        set_error("unsupported: %s", "tensor-core kernel needs N % 128 == 0, K % 128 == 0, 16-byte aligned a and b_packed");
         return W4A16_ERR_UNSUPPORTED;
     }
     // The documented contract: a workspace of at least what the size query advertises for these
