@@ -106,6 +106,20 @@ W4A16_API w4a16_status w4a16_load_ct(const void* ckpt_nk8, const void* scale_ng,
                                      void* stream);
 
 /*
+ * w4a16_gemm_kernel_choice — which kernel family w4a16_gemm runs for this shape and these
+ * pointers (W4A16_KERNEL_GEMV, W4A16_KERNEL_TC or W4A16_KERNEL_GEMV_FMA, the CUDA-core GEMV).
+ * Host only: no CUDA call, no device needed; the pointers are only checked for alignment and
+ * may be NULL (a NULL pointer counts as aligned).
+ *
+ *   M, N, K, group_size  as for w4a16_gemm.
+ *   a, b_packed, scales  the pointers w4a16_gemm would get, or NULL.
+ *   kernel               out: one of the W4A16_KERNEL_* values above.
+ * Errors: INVALID_ARG for a NULL `kernel` or a shape w4a16_gemm would reject.
+ */
+W4A16_API w4a16_status w4a16_gemm_kernel_choice(int64_t M, int64_t N, int64_t K, int32_t group_size, const void* a,
+                                                const void* b_packed, const void* scales, int32_t* kernel);
+
+/*
  * w4a16_gemm_workspace_bytes — bytes of device workspace w4a16_gemm needs for
  * this shape on the current device (0 when the shape needs none). Returns 0 for
  * shapes w4a16_gemm would reject. The value depends on the current device's SM

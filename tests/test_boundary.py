@@ -160,3 +160,44 @@ def test_python_binding_requires_cuda_tensors():
     a = torch.zeros(1, 256, dtype=torch.float16)
     with pytest.raises(TypeError):
         w.w4a16_gemm(a, torch.zeros(256, 8, dtype=torch.int32), torch.zeros(2, 64, dtype=torch.float16), None, 128)
+
+
+KERNELS = {"GEMV": 1, "TC": 2, "GEMV_FMA": 3}
+
+
+@pytest.mark.parametrize("M,N,K,G,ptrs,expect", [
+    (1, 14336, 4096, 128, {}, "GEMV"),
+    (16, 14336, 4096, 128, {}, "GEMV"),          # one GEMV launch
+    (17, 14336, 4096, 128, {}, "TC"),            # 112 column tiles >= 96
+    (32, 14336, 4096, 128, {}, "TC"),
+    (32, 6144, 4096, 128, {}, "GEMV"),           # 48 column tiles
+    (32, 12288, 4096, 128, {}, "TC"),            # exactly 96
+    (32, 12160, 4096, 128, {}, "GEMV"),          # 95
+    (33, 4096, 4096, 128, {}, "TC"),             # above 32 rows: the GEMM whenever it can
+    (64, 4096, 4160, 64, {}, "GEMV"),            # K % 128 != 0
+    (64, 4128, 4096, 128, {}, "GEMV"),           # N % 128 != 0, N % 32 == 0
+    (64, 4104, 4096, 128, {}, "GEMV_FMA"),       # N % 32 != 0
+    (1, 14336, 4096, 128, {"a": 0x10008}, "GEMV_FMA"),        # activations only 8-byte aligned
+    (64, 14336, 4096, 128, {"b": 0x20008}, "GEMV_FMA"),       # weights only 8-byte aligned
+    (64, 14336, 4096, 128, {"a": 0x10008}, "GEMV_FMA"),
+    (1, 14336, 4096, 128, {"s": 0x30004}, "GEMV_FMA"),        # scales only 4-byte aligned
+    (64, 14336, 4096, 128, {"s": 0x30004}, "TC"),             # the GEMM reads scales per element
+])
+def test_kernel_choice_table(M, N, K, G, ptrs, expect):
+    k = w.w4a16_gemm_kernel_choice(M, N, K, G, ptrs.get("a"), ptrs.get("b"), ptrs.get("s"))
+    assert k == KERNELS[expect]
+
+
+def test_kernel_choice_agrees_with_the_bench():
+    import bench
+    for M in (1, 8, 16, 17, 24, 32, 33, 64, 128):
+        for N in (4096, 6144, 12160, 12288, 14336, 28672):
+            k = w.w4a16_gemm_kernel_choice(M, N, 4096, 128)
+            assert (k == KERNELS["TC"]) == bench.uses_tc(M, N), (M, N)
+
+
+def test_kernel_choice_rejects_bad_arguments():
+    v = ctypes.c_int32()
+    assert w.lib.w4a16_gemm_kernel_choice(1, 64, 256, 128, None, None, None, None) == w.W4A16_ERR_INVALID_ARG
+    assert w.lib.w4a16_gemm_kernel_choice(1, 60, 256, 128, None, None, None, ctypes.byref(v)) == w.W4A16_ERR_INVALID_ARG
+    assert "N must be" in w.lib.w4a16_last_error().decode()

@@ -39,6 +39,8 @@ lib.w4a16_repack.argtypes = [_p, _p, _i64, _i64, _p]
 lib.w4a16_repack.restype = ctypes.c_int
 lib.w4a16_load_ct.argtypes = [_p, _p, _p, _i64, _i64, _i32, _p, _p, _p, _p]
 lib.w4a16_load_ct.restype = ctypes.c_int
+lib.w4a16_gemm_kernel_choice.argtypes = [_i64, _i64, _i64, _i32, _p, _p, _p, ctypes.POINTER(ctypes.c_int32)]
+lib.w4a16_gemm_kernel_choice.restype = ctypes.c_int
 lib.w4a16_gemm_workspace_bytes.argtypes = [_i64, _i64, _i64, _i32]
 lib.w4a16_gemm_workspace_bytes.restype = _sz
 lib.w4a16_gemm_ex_workspace_bytes.argtypes = [_i64, _i64, _i64, _i32, ctypes.POINTER(W4A16Options)]
@@ -59,7 +61,7 @@ lib.w4a16_status_string.restype = ctypes.c_char_p
 lib.w4a16_last_error.argtypes = []
 lib.w4a16_last_error.restype = ctypes.c_char_p
 
-EXPORTED = ("w4a16_repack", "w4a16_load_ct", "w4a16_gemm_workspace_bytes", "w4a16_gemm", "w4a16_gemm_ex_workspace_bytes",
+EXPORTED = ("w4a16_repack", "w4a16_load_ct", "w4a16_gemm_kernel_choice", "w4a16_gemm_workspace_bytes", "w4a16_gemm", "w4a16_gemm_ex_workspace_bytes",
             "w4a16_gemm_ex", "w4a16_workspace_status", "w4a16_status_string", "w4a16_last_error",
             "w4a16_gemm_noalloc", "w4a16_noalloc_scratch_bytes")
 
@@ -101,6 +103,19 @@ def _opts(kernel, split_k, debug_flags=0, wait_limit_us=0, launch_flags=0):
 
 def w4a16_status_string(status: int) -> str:
     return lib.w4a16_status_string(int(status)).decode()
+
+
+def w4a16_gemm_kernel_choice(M: int, N: int, K: int, group_size: int, a=None, b_packed=None, scales=None) -> int:
+    """The kernel family w4a16_gemm runs (KERNEL_GEMV, KERNEL_TC or KERNEL_GEMV_FMA); host only.
+    Pointers may be given as tensors, integers or None (None counts as aligned)."""
+    def ptr(x):
+        if x is None:
+            return None
+        return ctypes.c_void_p(x.data_ptr() if isinstance(x, torch.Tensor) else int(x))
+    k = ctypes.c_int32()
+    _check(lib.w4a16_gemm_kernel_choice(M, N, K, group_size, ptr(a), ptr(b_packed), ptr(scales), ctypes.byref(k)),
+           "w4a16_gemm_kernel_choice")
+    return int(k.value)
 
 
 def w4a16_gemm_workspace_bytes(M: int, N: int, K: int, group_size: int, kernel=None, split_k: int = 0) -> int:

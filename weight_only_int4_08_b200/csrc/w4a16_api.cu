@@ -249,6 +249,22 @@ size_t w4a16_gemm_ex_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t gr
     return ws_bound(M, N, K, group_size, opts, sms);
 }
 
+w4a16_status w4a16_gemm_kernel_choice(int64_t M, int64_t N, int64_t K, int32_t group_size, const void* a,
+                                      const void* b_packed, const void* scales, int32_t* kernel) {
+    g_last_error[0] = 0;
+    if (!kernel) return fail_arg("NULL pointer");
+    if (const char* why = check_gemm_shape(M, N, K, group_size)) return fail_arg(why);
+    const void* pa = a ? a : (const void*)16;
+    const void* pb = b_packed ? b_packed : (const void*)16;
+    const void* ps = scales ? scales : (const void*)16;
+    // the same decisions as choose() and the launch path, without the device queries
+    if (auto_prefers_tc(M, N) && tc_supported(M, N, K, group_size, pa, pb))
+        *kernel = W4A16_KERNEL_TC;
+    else
+        *kernel = gemv_mma_supported(N, K, pa, pb, ps) ? W4A16_KERNEL_GEMV : W4A16_KERNEL_GEMV_FMA;
+    return W4A16_OK;
+}
+
 size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t group_size) {
     return w4a16_gemm_ex_workspace_bytes(M, N, K, group_size, nullptr);
 }
