@@ -32,6 +32,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -97,11 +98,11 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        fd, self.path = tempfile.mkstemp(prefix=f"w4a16_clocks_rank{index}_", suffix=".csv")
+        os.close(fd)
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -123,6 +124,10 @@ class ClockSampler:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
                 rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not rows:
             return None
         sm = [float(r[1]) for r in rows]
@@ -288,6 +293,10 @@ def run_gpu(args):
     g_main = capture(torch, prob.step, chunk)
     tail = K_steps % chunk
     g_tail = capture(torch, prob.step, tail) if tail else None
+    # The first replay of a graph uploads it to the device; do that outside the timed region.
+    g_main.replay()
+    if g_tail is not None:
+        g_tail.replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -494,6 +503,19 @@ def run_stack(torch, w, peaks):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
+def host_cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's processor string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown CPU"
+
+
 def cpu_baseline(case, seconds=10.0):
     import oracle
     oracle.gemm(case["a"], case["b"], case["s"], case["z"], case["G"], case["zp_bias"])  # load/build
@@ -507,7 +529,7 @@ def cpu_baseline(case, seconds=10.0):
     byts = alg_bytes(case["M"], case["K"], case["N"], case["G"], case["z"] is not None)
     return {"value": round(byts / dt / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{n} full GEMMs of the M=1 K=4096 N=14336 workload, {dt * 1e3:.1f} ms each, 1 thread "
-                      f"of {os.cpu_count()} host cores"}
+                      f"of {os.cpu_count()} host cores ({host_cpu_model()})"}
 
 
 def run_reference(args):
@@ -533,7 +555,8 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32 (CPU oracle)",
             "data": "synthetic", "config": {"workload": "decode GEMV M=1 K=4096 N=14336 G=128 sym zp_bias=8 (8B MLP-up shape)"},
             "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{steps} full GEMMs of the workload on 1 of {os.cpu_count()} host cores"},
+                             "sample": f"{steps} full GEMMs of the workload on 1 of {os.cpu_count()} host cores "
+                                       f"({host_cpu_model()})"},
             "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

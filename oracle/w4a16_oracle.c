@@ -21,7 +21,7 @@
  * the same page: checkpoint layout [N, K/8] (8 nibbles per int32 along K) to
  * kernel layout [K, N/8] (8 nibbles per int32 along N).
  *
- * Readings where the page is silent (each listed in the design doc):
+ * Readings taken where the page is silent:
  *   - nibble j of a 32-bit word (bits 4j..4j+3) holds the element with index
  *     8*c + j along the packed dimension, for weights, zeros and checkpoint;
  *   - nibbles are unsigned 0..15;
