@@ -180,8 +180,9 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  *     GEMV_FMA forces the CUDA-core fp32 loop;
  *     TC forces the tensor-core GEMM (any M; UNSUPPORTED when the shape or
  *     alignment rules above fail).
- *   split_k: 0 = automatic, else the number of K slices (1..256) the kernel
- *     splits its work into (the tensor-core GEMM clamps it to K/64).
+ *   split_k: 0 = automatic, else (1..1024) the number of K slices the kernel
+ *     splits its work into: the tensor-core GEMM clamps it to K/128, the
+ *     mma.sync GEMV to a thread-block cluster (at most 4 CTAs per column tile).
  *   debug_flags: 0 in normal use. W4A16_DEBUG_STALL_LOADS makes the kernels'
  *     load issuers issue nothing, so every device-side wait runs out: the call
  *     then leaves W4A16_ERR_TIMEOUT in the workspace status word (read it with
@@ -236,11 +237,14 @@ W4A16_API w4a16_status w4a16_workspace_status(void* workspace, int32_t clear, in
  * Some callers cannot hand over a workspace: code that must not call cudaMalloc
  * because it can synchronise the whole device in the middle of a latency-
  * critical loop, or code embedded in a program whose device memory belongs to
- * another allocator. This variant runs the CUDA-core GEMV kernel family (any M;
- * M > 8 in 8-row blocks) with its scratch memory — status word, split-K
- * counters and fp32 partials — in a fixed array compiled into the library
- * (w4a16_noalloc_scratch_bytes() bytes, 8 MiB) instead of a workspace. It
- * allocates nothing and calls no allocating routine.
+ * another allocator. This variant runs the GEMV kernel family with its scratch
+ * memory (status word, split-K arrival counters and fp32 partials) in a fixed
+ * array compiled into the library (w4a16_noalloc_scratch_bytes() bytes, 8 MiB)
+ * instead of a workspace. It allocates nothing and calls no allocating routine.
+ * Which GEMV runs follows the GEMV rule of w4a16_gemm_ex: the warp mma.sync GEMV
+ * (16 rows of A per launch) when N % 32 == 0, a and b_packed are 16-byte and
+ * scales 8-byte aligned; otherwise the CUDA-core split-K GEMV (8 rows per
+ * launch), whose arrival counters and partials live in the array.
  *
  *   Arguments a .. out and stream: as for w4a16_gemm (no workspace arguments).
  *   Limit: a shape whose GEMV scratch need exceeds the fixed array returns
@@ -249,8 +253,11 @@ W4A16_API w4a16_status w4a16_workspace_status(void* workspace, int32_t clear, in
  *   The first call on a device looks up the array's device address with that
  *     device current (cudaGetSymbolAddress) and caches it; make that first call
  *     before any stream capture.
- *   Each call first clears the array's status word and counters on `stream`
- *     (cudaMemsetAsync), then launches the kernel on `stream`.
+ *   Each call first clears the part of the array it uses beyond the status
+ *     word (split-K counters, partial sums) on `stream` (cudaMemsetAsync), then
+ *     launches the kernel on `stream`. The status word is not cleared by calls:
+ *     a device-side timeout stays recorded until w4a16_noalloc_status reads and
+ *     clears it.
  *   All calls share the one array: calls that overlap on the GPU (different
  *     streams without ordering, or several host threads) race and give wrong
  *     results. Order them on one stream or with events.
@@ -259,6 +266,27 @@ W4A16_API w4a16_status w4a16_workspace_status(void* workspace, int32_t clear, in
 W4A16_API w4a16_status w4a16_gemm_noalloc(const void* a, const void* b_packed, const void* scales,
                                           const void* qzeros, int64_t M, int64_t N, int64_t K, int32_t group_size,
                                           int32_t zp_bias, void* out, void* stream);
+
+/*
+ * w4a16_gemm_noalloc with options (NULL opts = w4a16_gemm_noalloc). Same contract.
+ * opts->kernel may be W4A16_KERNEL_AUTO or W4A16_KERNEL_GEMV (the GEMV rule above)
+ * or W4A16_KERNEL_GEMV_FMA (the CUDA-core split-K GEMV); W4A16_KERNEL_TC returns
+ * W4A16_ERR_INVALID_ARG. The other fields as for w4a16_gemm_ex.
+ */
+W4A16_API w4a16_status w4a16_gemm_noalloc_ex(const void* a, const void* b_packed, const void* scales,
+                                             const void* qzeros, int64_t M, int64_t N, int64_t K,
+                                             int32_t group_size, int32_t zp_bias, void* out, void* stream,
+                                             const w4a16_gemm_options* opts);
+
+/*
+ * w4a16_noalloc_status — read the status word of the fixed scratch array of the
+ * current device into *status (W4A16_OK, or W4A16_ERR_TIMEOUT when a bounded
+ * device-side wait of a no-allocation call gave up; that call's output is then
+ * undefined). Synchronises `stream`. Pass clear != 0 to reset the word to
+ * W4A16_OK after reading.
+ * Errors: INVALID_ARG for a NULL `status`; CUDA for a failed lookup or copy.
+ */
+W4A16_API w4a16_status w4a16_noalloc_status(int32_t clear, int32_t* status, void* stream);
 
 /* Size in bytes of the fixed scratch array used by w4a16_gemm_noalloc. */
 W4A16_API size_t w4a16_noalloc_scratch_bytes(void);

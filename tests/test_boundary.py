@@ -124,7 +124,7 @@ def test_options_are_checked():
     o = w.W4A16Options(7, 0)
     rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
     assert rc == w.W4A16_ERR_INVALID_ARG
-    o = w.W4A16Options(1, 999)
+    o = w.W4A16Options(1, 1025)
     rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
     assert rc == w.W4A16_ERR_INVALID_ARG
     o = w.W4A16Options(0, 0, 0, 0, 2)   # an undefined launch flag
@@ -201,3 +201,18 @@ def test_kernel_choice_rejects_bad_arguments():
     assert w.lib.w4a16_gemm_kernel_choice(1, 64, 256, 128, None, None, None, None) == w.W4A16_ERR_INVALID_ARG
     assert w.lib.w4a16_gemm_kernel_choice(1, 60, 256, 128, None, None, None, ctypes.byref(v)) == w.W4A16_ERR_INVALID_ARG
     assert "N must be" in w.lib.w4a16_last_error().decode()
+
+
+def test_noalloc_checks_on_host():
+    """The no-allocation GEMM refuses bad arguments and the tensor-core kernel before any CUDA
+    call (its scratch bound covers the GEMV family only); its status query needs a pointer."""
+    v = ctypes.c_int32()
+    assert w.lib.w4a16_noalloc_status(0, None, None) == w.W4A16_ERR_INVALID_ARG
+    args = (GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None)
+    assert w.lib.w4a16_gemm_noalloc(None, *args[1:]) == w.W4A16_ERR_INVALID_ARG
+    assert w.lib.w4a16_gemm_noalloc(*args[:8], 16, *args[9:]) == w.W4A16_ERR_INVALID_ARG   # zp_bias > 15
+    tc = w.W4A16Options(w.KERNEL_TC, 0, 0, 0, 0)
+    assert w.lib.w4a16_gemm_noalloc_ex(*args, ctypes.byref(tc)) == w.W4A16_ERR_INVALID_ARG
+    assert "GEMV kernels only" in w.lib.w4a16_last_error().decode()
+    assert int(w.lib.w4a16_noalloc_scratch_bytes()) == 8 << 20
+    del v

@@ -54,6 +54,11 @@ lib.w4a16_workspace_status.argtypes = [_p, _i32, ctypes.POINTER(ctypes.c_int32),
 lib.w4a16_workspace_status.restype = ctypes.c_int
 lib.w4a16_gemm_noalloc.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _i32, _p, _p]
 lib.w4a16_gemm_noalloc.restype = ctypes.c_int
+lib.w4a16_gemm_noalloc_ex.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _i32, _i32, _p, _p,
+                                      ctypes.POINTER(W4A16Options)]
+lib.w4a16_gemm_noalloc_ex.restype = ctypes.c_int
+lib.w4a16_noalloc_status.argtypes = [_i32, ctypes.POINTER(ctypes.c_int32), _p]
+lib.w4a16_noalloc_status.restype = ctypes.c_int
 lib.w4a16_noalloc_scratch_bytes.argtypes = []
 lib.w4a16_noalloc_scratch_bytes.restype = _sz
 lib.w4a16_status_string.argtypes = [ctypes.c_int]
@@ -63,7 +68,7 @@ lib.w4a16_last_error.restype = ctypes.c_char_p
 
 EXPORTED = ("w4a16_repack", "w4a16_load_ct", "w4a16_gemm_kernel_choice", "w4a16_gemm_workspace_bytes", "w4a16_gemm", "w4a16_gemm_ex_workspace_bytes",
             "w4a16_gemm_ex", "w4a16_workspace_status", "w4a16_status_string", "w4a16_last_error",
-            "w4a16_gemm_noalloc", "w4a16_noalloc_scratch_bytes")
+            "w4a16_gemm_noalloc", "w4a16_gemm_noalloc_ex", "w4a16_noalloc_status", "w4a16_noalloc_scratch_bytes")
 
 
 class W4A16Error(RuntimeError):
@@ -229,6 +234,13 @@ def w4a16_gemm_noalloc(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Te
     _check(lib.w4a16_gemm_noalloc(pa, pb, ps, pz, M, N, K, group_size, zp_bias, po, _stream_ptr(stream)),
            "w4a16_gemm_noalloc")
     return out
+
+
+def w4a16_noalloc_status(clear: bool = False, stream=None) -> int:
+    """Status word of the no-allocation GEMM's fixed scratch array (synchronises the stream)."""
+    v = ctypes.c_int32(-1)
+    _check(lib.w4a16_noalloc_status(int(clear), ctypes.byref(v), _stream_ptr(stream)), "w4a16_noalloc_status")
+    return int(v.value)
 
 
 def w4a16_workspace_status(workspace: torch.Tensor, clear: bool = False, stream=None) -> int:

@@ -57,8 +57,8 @@ GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_reque
                    bool tma_ok);
 
 // The stream-K mma.sync GEMV: N % 32 == 0, 16-byte aligned weights and activations,
-// 8-byte aligned scales.
-bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s);
+// 8-byte aligned scales (z, the zeros, may be NULL; 4-byte alignment suffices).
+bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s, const void* z);
 GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count);
 cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M,
                             int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace,

@@ -674,7 +674,8 @@ SkLayout sk_layout(int mt, int64_t N, int64_t K, int split_k_request, int sm_cou
 
 }  // namespace
 
-bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s) {
+bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s, const void* z) {
+    (void)z;   // zeros are read with 4-byte copies
     const int64_t units = (N + kTileN - 1) / kTileN * ((K + 63) / 64);   // counted in 32 bits (64-row units at most)
     return N % 32 == 0 && units < ((int64_t)1 << 31) && (reinterpret_cast<uintptr_t>(b) % 16) == 0 &&
            (reinterpret_cast<uintptr_t>(a) % 16) == 0 && (reinterpret_cast<uintptr_t>(s) % 8) == 0;

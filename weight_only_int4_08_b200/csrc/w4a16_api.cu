@@ -96,7 +96,7 @@ bool auto_prefers_tc(int64_t M, int64_t N) {
     return M > kGemvMaxM || (M > kGemvOneLaunchM && N / 128 >= kTcMinTiles);
 }
 Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms,
-              const void* a, const void* b, const void* s) {
+              const void* a, const void* b, const void* s, const void* z) {
     Choice c{};
     const int req = opts ? opts->kernel : W4A16_KERNEL_AUTO;
     const bool tc_ok = tc_supported(M, N, K, G, a ? a : (const void*)16, b ? b : (const void*)16);
@@ -107,7 +107,7 @@ Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_optio
     if (c.kernel == W4A16_KERNEL_TC) {
         if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, split);
     } else if (req != W4A16_KERNEL_GEMV_FMA &&
-               gemv_mma_supported(N, K, a ? a : (const void*)16, b ? b : (const void*)16, s ? s : (const void*)16)) {
+               gemv_mma_supported(N, K, a ? a : (const void*)16, b ? b : (const void*)16, s ? s : (const void*)16, z)) {
         c.gemv = plan_gemv_mma(M, N, K, G, split, sms);
     } else {
         c.gemv = plan_gemv(M, N, K, G, split, sms, b ? max_vec_for(b) : 4, true);
@@ -261,7 +261,7 @@ w4a16_status w4a16_gemm_kernel_choice(int64_t M, int64_t N, int64_t K, int32_t g
     if (auto_prefers_tc(M, N) && tc_supported(M, N, K, group_size, pa, pb))
         *kernel = W4A16_KERNEL_TC;
     else
-        *kernel = gemv_mma_supported(N, K, pa, pb, ps) ? W4A16_KERNEL_GEMV : W4A16_KERNEL_GEMV_FMA;
+        *kernel = gemv_mma_supported(N, K, pa, pb, ps, nullptr) ? W4A16_KERNEL_GEMV : W4A16_KERNEL_GEMV_FMA;
     return W4A16_OK;
 }
 
@@ -279,7 +279,7 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
     if (!qzeros && (zp_bias < 0 || zp_bias > 15)) return fail_arg("zp_bias must be in 0..15");
     if (opts && (opts->kernel < W4A16_KERNEL_AUTO || opts->kernel > W4A16_KERNEL_GEMV_FMA))
         return fail_arg("unknown kernel option");
-    if (opts && (opts->split_k < 0 || opts->split_k > 256)) return fail_arg("split_k must be in 0..256");
+    if (opts && (opts->split_k < 0 || opts->split_k > 1024)) return fail_arg("split_k must be in 0..1024");
     if (opts && (opts->debug_flags & ~(uint32_t)W4A16_DEBUG_STALL_LOADS)) return fail_arg("unknown debug flag");
     if (opts && (opts->launch_flags & ~(uint32_t)W4A16_LAUNCH_PDL)) return fail_arg("unknown launch flag");
     if (!aligned(a, 2) || !aligned(scales, 2) || !aligned(out, 2)) return fail_arg("fp16 pointers must be 2-byte aligned");
@@ -297,7 +297,7 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
         set_error("unsupported: %s", "this library is built for sm_100 (B200) devices");
         return W4A16_ERR_UNSUPPORTED;
     }
-    Choice c = choose(M, N, K, group_size, opts, sms, a, b_packed, scales);
+    Choice c = choose(M, N, K, group_size, opts, sms, a, b_packed, scales, qzeros);
     if (c.kernel == W4A16_KERNEL_TC && !tc_supported(M, N, K, group_size, a, b_packed)) {
         set_error("unsupported: %s", "tensor-core kernel needs N % 128 == 0, K % 128 == 0, 16-byte aligned a and b_packed");
         return W4A16_ERR_UNSUPPORTED;
