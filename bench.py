@@ -491,13 +491,28 @@ def run_stack(torch, w, peaks):
         g = capture(torch, one_pass, 1)
         time_graph(torch, g, 2)
         t = time_graph(torch, g, 10) / 10
+        del g
+        # Gap analysis: each linear alone, its 32 layers back to back (the same calls as in the pass);
+        # t_sum is what the pass would take if the four shapes cost what they cost alone.
+        per_linear = {}
+        for idx, name in enumerate(("qkv", "o", "gate_up", "down")):
+            def one_linear(idx=idx):
+                for row in layers:
+                    b, s, k, n = row[idx]
+                    w.w4a16_gemm(acts[0][idx], b, s, None, 128, 8, out=outs[idx], workspace=wss[idx], pdl=True)
+            gl = capture(torch, one_linear, 1)
+            time_graph(torch, gl, 2)
+            per_linear[name] = time_graph(torch, gl, 10) / 10 / synth.N_LAYERS
+            del gl
+        t_sum = synth.N_LAYERS * sum(per_linear.values())
         byts = sum(alg_bytes(M, k, n, 128, False) for row in layers for (_, _, k, n) in row)
         flops = sum(alg_flops(M, k, n) for row in layers for (_, _, k, n) in row)
         t_roof = max(byts / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
         res[f"config5_stack_M{M}"] = {"us": round(t * 1e6, 1), "GB/s": round(byts / t / 1e9, 1),
                                       "TFLOP/s": round(flops / t / 1e12, 2), "roofline_us": round(t_roof * 1e6, 1),
-                                      "frac_of_roofline": round(t_roof / t, 4), "launches": 128}
-        del g
+                                      "frac_of_roofline": round(t_roof / t, 4), "launches": 128,
+                                      "t_sum_us": round(t_sum * 1e6, 1),
+                                      "per_linear_us": {k: round(v * 1e6, 2) for k, v in per_linear.items()}}
     return res
 
 

@@ -74,6 +74,9 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 #define W4A16_WAIT_SLEEP_NS 20000  // suspend hint of the polling try_wait (0: no hint)
 #endif
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+    // A phase that has completed is seen by the non-blocking test, without the potentially
+    // suspending try_wait.
+    if (mbar_test_wait(bar, parity)) return true;
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
