@@ -72,19 +72,35 @@ constexpr int kTmemStages = 4;                  // A slots in TMEM
 // the epilogue need the registers that more threads would take. A group's stage ends with a
 // wait for its TMEM stores; a second group keeps another stage in flight meanwhile.
 __host__ __device__ constexpr int deq_warps(int mn) { return mn <= 64 ? 8 : 4; }
-__host__ __device__ constexpr int tc_threads(int mn) { return (deq_warps(mn) + 6) * 32; }
+// Weight producers: stage i of the weight ring is issued by producer i % P (one: measured on
+// B200 at M = 32, four issuing warps did not raise the weight rate).
+__host__ __device__ constexpr int wproducer_warps(int mn) { return (void)mn, 1; }
+// Warps: dequantisers, weight producers, an activation producer, the MMA issuer, four epilogue warps.
+__host__ __device__ constexpr int tc_threads(int mn) { return (deq_warps(mn) + wproducer_warps(mn) + 6) * 32; }
 
 template <int MN>
 struct TcCfg {
-    // a multiple of kTmemStages (the unrolled issue loop relies on it)
-    static constexpr int kSmemStages = MN <= 64 ? 8 : 4;
+    // Weights and activations have rings of their own. A weight slot is free again as soon as its
+    // dequantiser group has read it; an activation slot only when the stage's MMAs have completed.
+    // Measured on B200 (M = 32, per-stage timeline): with one ring released by the MMA commit, a
+    // slot was busy ~1.3 us after its data landed and a refill took ~2.85 us to land, which set
+    // the stage rate (12 slots per ~4.1 us).
+    static constexpr int kAStages = MN <= 48 ? 8 : 4;   // a multiple of kTmemStages (unrolled MMA loop)
     static constexpr int kBoxBytes = MN * kBoxK * 2;        // one activation box: MN rows x 128 B
     static constexpr int kBStageBytes = kBoxes * kBoxBytes;
+    static constexpr int kWStagesFit = (200 * 1024 - kAStages * kBStageBytes) / kWStageBytes;
+    static constexpr int kWStages = (kWStagesFit > 16 ? 16 : kWStagesFit) / wproducer_warps(MN) * wproducer_warps(MN);
+    // Accumulator buffers in TMEM: the MMAs of segment g + kDBufs wait for the epilogue to have read
+    // segment g. Measured on B200 (M = 32, per-stage timeline): with two buffers that round trip
+    // (MMA completion, commit, epilogue read-out) set the stage rate at ~0.45 us, the MMA warp
+    // running ~1.2 us behind the dequantisers; the columns left after the A slots allow more.
+    static constexpr int kDBufs = MN <= 32 ? 8 : MN <= 64 ? 4 : 2;
     static constexpr int kDCol = kTmemStages * kAColsPerStage;   // first accumulator column
-    static constexpr int kColsNeeded = kDCol + 2 * MN;
+    static constexpr int kColsNeeded = kDCol + kDBufs * MN;
     static constexpr int kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64 : kColsNeeded <= 128 ? 128
                                    : kColsNeeded <= 256 ? 256 : 512;
-    static constexpr size_t kSmemBytes = 1024 /*align slack*/ + (size_t)kSmemStages * (kBStageBytes + kWStageBytes);
+    static constexpr size_t kSmemBytes = 1024 /*align slack*/ + (size_t)kAStages * kBStageBytes +
+                                         (size_t)kWStages * kWStageBytes;
 };
 
 struct TcArgs {
@@ -136,17 +152,22 @@ __global__ void __launch_bounds__(tc_threads(MN), 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap, TcArgs p) {
     using C = TcCfg<MN>;
     constexpr int kDeqWarps = deq_warps(MN);
-    constexpr int kProducerWarp = kDeqWarps, kMmaWarp = kDeqWarps + 1, kEpiWarp0 = kDeqWarps + 2;
-    constexpr int SS = C::kSmemStages;
+    constexpr int kWProducers = wproducer_warps(MN);
+    constexpr int kWProducer = kDeqWarps, kAProducer = kDeqWarps + kWProducers, kMmaWarp = kAProducer + 1,
+                  kEpiWarp0 = kMmaWarp + 1;
+    constexpr int WS = C::kWStages, AS = C::kAStages;
+    static_assert(WS % kWProducers == 0, "every weight slot has one producer");
     extern __shared__ __align__(1024) unsigned char s_raw[];
     unsigned char* s_base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(s_raw) + 1023) & ~(uintptr_t)1023);
-    unsigned char* s_b = s_base;                                   // [SS][2][MN x 128 B], 1024-aligned boxes
-    unsigned char* s_w = s_base + (size_t)SS * C::kBStageBytes;    // [SS][128 rows x 64 B], 1024-aligned stages
+    unsigned char* s_b = s_base;                                   // [AS][2][MN x 128 B], 1024-aligned boxes
+    unsigned char* s_w = s_base + (size_t)AS * C::kBStageBytes;    // [WS][128 rows x 64 B], 1024-aligned stages
 
-    __shared__ __align__(8) uint64_t bar_full[SS], bar_empty[SS];
+    // weight ring (TMA / dequantiser group) and activation ring (TMA / MMA commit)
+    __shared__ __align__(8) uint64_t bar_wfull[WS], bar_wempty[WS], bar_full[AS], bar_empty[AS];
     __shared__ __align__(8) uint64_t bar_afull[kTmemStages], bar_aempty[kTmemStages];
-    __shared__ __align__(8) uint64_t bar_dfull[2], bar_dempty[2], bar_drain;
+    constexpr int DB = C::kDBufs;
+    __shared__ __align__(8) uint64_t bar_dfull[DB], bar_dempty[DB], bar_drain;
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
     __shared__ int s_last;
@@ -160,7 +181,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 
     if (threadIdx.x == 0) {
         s_abort = 0;
-        for (int i = 0; i < SS; ++i) {
+        for (int i = 0; i < WS; ++i) {
+            ptx::mbar_init(ptx::smem_addr(&bar_wfull[i]), 1);
+            ptx::mbar_init(ptx::smem_addr(&bar_wempty[i]), 4);   // the four warps of a dequantiser group
+        }
+        for (int i = 0; i < AS; ++i) {
             ptx::mbar_init(ptx::smem_addr(&bar_full[i]), 1);
             ptx::mbar_init(ptx::smem_addr(&bar_empty[i]), 1);
         }
@@ -168,7 +193,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             ptx::mbar_init(ptx::smem_addr(&bar_afull[i]), 128);   // one group of four warps per stage
             ptx::mbar_init(ptx::smem_addr(&bar_aempty[i]), 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < DB; ++i) {
             ptx::mbar_init(ptx::smem_addr(&bar_dfull[i]), 1);
             ptx::mbar_init(ptx::smem_addr(&bar_dempty[i]), 128);
         }
@@ -184,25 +209,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     ptx::tc_fence_after();
     const uint32_t tmem = s_tmem;
 
-    if (warp == kProducerWarp) {
-        // ------------------------------------------------------------ producer
-        // Converged loop, one elected lane issuing (as for the MMA warp).
+    if (warp == kAProducer) {
+        // ------------------------------------------------- activation producer
+        // The activation ring, in stage order: two 2-D TMA boxes per stage (MN rows x 64 k each,
+        // 128-byte swizzle, rows past M read as zero). Converged loop, one elected lane issuing.
         const bool leader = ptx::elect_one();
-        if (leader) {
-            ptx::prefetch_tensormap(&amap);
-            ptx::prefetch_tensormap(&wmap);
-        }
-        const uint32_t tx = kWStageBytes + C::kBStageBytes;
+        if (leader) ptx::prefetch_tensormap(&amap);
         int issued = 0;
         for (int i = 0; i < nst && !p.stall_loads; ++i) {
-            const int s = i % SS;
-            const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_empty[s]), ((i / SS) & 1) ^ 1, &s_abort, p.wait_ns);
+            const int s = i % AS;
+            const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_empty[s]), ((i / AS) & 1) ^ 1, &s_abort, p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) break;
             if (leader) {
                 const uint32_t full = ptx::smem_addr(&bar_full[s]);
-                ptx::mbar_arrive_expect_tx(full, tx);
+                ptx::mbar_arrive_expect_tx(full, (uint32_t)C::kBStageBytes);
                 const int32_t k0 = (int32_t)((st_lo + i) * kStageK);
-                ptx::tma_load_2d(ptx::smem_addr(s_w + (size_t)s * kWStageBytes), &wmap, tile * kTileWords, k0, full);
 #pragma unroll
                 for (int x = 0; x < kBoxes; ++x)
                     ptx::tma_load_2d(ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes + x * C::kBoxBytes), &amap,
@@ -213,8 +234,38 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         }
         if (s_abort && leader) {  // let copies already issued land before the CTA leaves
             volatile int dummy = 0;
-            for (int i = max(0, issued - SS); i < issued; ++i)
-                ptx::mbar_wait(ptx::smem_addr(&bar_full[i % SS]), (i / SS) & 1, &dummy, p.wait_ns);
+            for (int i = max(0, issued - AS); i < issued; ++i)
+                ptx::mbar_wait(ptx::smem_addr(&bar_full[i % AS]), (i / AS) & 1, &dummy, p.wait_ns);
+        }
+    } else if (warp >= kWProducer && warp < kAProducer) {
+        // ------------------------------------------------------------ weight producers
+        // Weight producer p streams weight stages p, p + P, ... Converged loops, one elected lane
+        // issuing (as for the MMA warp).
+        const int R = WS;
+        const int first = warp - kWProducer, step = kWProducers;
+        uint64_t* fullb = bar_wfull;
+        uint64_t* emptyb = bar_wempty;
+        const bool leader = ptx::elect_one();
+        if (leader) ptx::prefetch_tensormap(&wmap);
+        const uint32_t tx = (uint32_t)kWStageBytes;
+        int issued = -1;   // last stage this warp issued
+        for (int i = first; i < nst && !p.stall_loads; i += step) {
+            const int s = i % R;
+            const bool okw = ptx::mbar_wait(ptx::smem_addr(&emptyb[s]), ((i / R) & 1) ^ 1, &s_abort, p.wait_ns);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            if (leader) {
+                const uint32_t full = ptx::smem_addr(&fullb[s]);
+                ptx::mbar_arrive_expect_tx(full, tx);
+                const int32_t k0 = (int32_t)((st_lo + i) * kStageK);
+                ptx::tma_load_2d(ptx::smem_addr(s_w + (size_t)s * kWStageBytes), &wmap, tile * kTileWords, k0, full);
+            }
+            __syncwarp();
+            issued = i;
+        }
+        if (s_abort && leader) {  // let copies already issued land before the CTA leaves
+            volatile int dummy = 0;
+            for (int i = issued; i >= 0 && i > issued - R; i -= step)
+                ptx::mbar_wait(ptx::smem_addr(&fullb[i % R]), (i / R) & 1, &dummy, p.wait_ns);
         }
     } else if (warp < kDeqWarps) {
         // -------------------------------------------------------- dequantisers
@@ -270,9 +321,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             }
         }
         for (int i = dg; i < nst; i += kDeqGroups) {
-            const int s = i % SS, ts = i % kTmemStages;
-            // Wait outcomes are made warp-uniform: the tcgen05 stores below are .sync.aligned.
-            bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns);
+            const int s = i % WS, ts = i % kTmemStages;
+            // Wait outcomes are made warp-uniform: the tcgen05 stores below are .sync.aligned. The
+            // stage's activations are waited for here too, so that the MMA warp's one wait (for the
+            // TMEM slot) also orders the activation tile before its MMAs.
+            bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_wfull[s]), (i / WS) & 1, &s_abort, p.wait_ns);
+            okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_full[i % AS]), (i / AS) & 1, &s_abort, p.wait_ns);
             okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_aempty[ts]), ((i / kTmemStages) & 1) ^ 1, &s_abort,
                                         p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) break;
@@ -307,6 +361,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 const uint32_t col = (uint32_t)(ts * kAColsPerStage + 16 * hh);
                 ptx::tmem_st_16x128b_x4(lane_base + col, lo);
                 ptx::tmem_st_16x128b_x4(lane_base + (16u << 16) + col, hi);
+                if (hh == kStageK / 32 - 1) {
+                    // the weight stage is read: its slot can be refilled
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&bar_wempty[s]));
+                }
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -327,23 +386,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             const uint64_t bdesc0 = kmajor_sw128_desc(ptx::smem_addr(s_b));
             const uint32_t t_d = tmem + (uint32_t)C::kDCol;
             bool ok = true;
-            for (int i0 = 0; i0 < nst && ok; i0 += SS) {
+            for (int i0 = 0; i0 < nst && ok; i0 += AS) {
 #pragma unroll
-                for (int u = 0; u < SS; ++u) {
+                for (int u = 0; u < AS; ++u) {
                     const int i = i0 + u;
                     if (i >= nst) break;
                     constexpr int kTsMask = kTmemStages - 1;
                     const int ts = u & kTsMask;
                     const bool seg_start = rem == gs || i == 0;
                     const bool seg_end = rem == 1 || i == nst - 1;
-                    const int db = sg & 1;
+                    const int db = sg % DB;
                     // The stage's A slot is complete only after every thread of its dequantiser group
                     // has waited for the stage's TMA barrier, so this wait also orders the activation
                     // tile before the MMAs (a second wait on that barrier cost ~150 cycles per stage).
                     bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort,
                                               p.wait_ns);
                     if (seg_start)
-                        okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1, &s_abort,
+                        okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg / DB) & 1) ^ 1, &s_abort,
                                                     p.wait_ns);
                     if (!__all_sync(0xffffffffu, okw)) {
                         ok = false;
@@ -379,9 +438,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             int64_t seg_next = (seg.k_lo / p.G + 1) * p.G;   // next group boundary after the slab start
             bool starts = true;
             for (int i = 0; i < nst; ++i) {
-                const int s = i % SS, ts = i % kTmemStages;
+                const int s = i % AS, ts = i % kTmemStages;
                 bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_afull[ts]), (i / kTmemStages) & 1, &s_abort, p.wait_ns);
-                okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / SS) & 1, &s_abort, p.wait_ns);
+                okw = okw && ptx::mbar_wait(ptx::smem_addr(&bar_full[s]), (i / AS) & 1, &s_abort, p.wait_ns);
                 if (!__all_sync(0xffffffffu, okw)) break;
                 ptx::tc_fence_after();
                 const uint32_t bbase = ptx::smem_addr(s_b + (size_t)s * C::kBStageBytes);
@@ -389,11 +448,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 #pragma unroll
                 for (int j = 0; j < kMmaPerStage; ++j) {
                     const int64_t k = (st_lo + i) * kStageK + 16 * j;
-                    const int db = sg & 1;
+                    const int db = sg % DB;
                     const bool ends = k + 16 == seg.k_hi || k + 16 == seg_next;
                     if (k + 16 == seg_next) seg_next += p.G;
                     if (starts) {
-                        const bool okd = ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg >> 1) & 1) ^ 1,
+                        const bool okd = ptx::mbar_wait(ptx::smem_addr(&bar_dempty[db]), ((sg / DB) & 1) ^ 1,
                                                         &s_abort, p.wait_ns);
                         if (!__all_sync(0xffffffffu, okd)) {
                             ok = false;
@@ -455,8 +514,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             sc1 = sc2;
             sc2 = sc3;
             sc3 = scale_of(g_idx + 4);
-            const int db = sg & 1;
-            const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_dfull[db]), (sg >> 1) & 1, &s_abort, p.wait_ns);
+            const int db = sg % DB;
+            const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_dfull[db]), (sg / DB) & 1, &s_abort, p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) {  // warp-uniform: tcgen05.ld is .sync.aligned
                 ok = false;
                 break;
@@ -572,7 +631,8 @@ int tc_ctas_per_sm(int mn) {
     const int by_smem = (int)((228 * 1024) / (smem + fa.sharedSizeBytes + 1024));
     const int regs_per_warp = (regs + 7) / 8 * 8 * 32;  // allocation granularity: 8 registers per thread
     const int by_regs = 65536 / (regs_per_warp * (tc_threads(mn) / 32));
-    const int cols = kTmemStages * kAColsPerStage + 2 * mn <= 256 ? 256 : 512;
+    const int dbufs = mn <= 32 ? 8 : mn <= 64 ? 4 : 2;   // TcCfg<MN>::kDBufs
+    const int cols = kTmemStages * kAColsPerStage + dbufs * mn <= 256 ? 256 : 512;
     n = std::max(1, std::min(std::min(by_smem, by_regs), 512 / cols));
     g_tc_occ[mn / 16].store(n, std::memory_order_relaxed);
     return n;
