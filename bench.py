@@ -164,19 +164,21 @@ class Problem:
         self.bs = [b0] + [b0.clone() for _ in range(copies - 1)]
         self.ss = [s0] + [s0.clone() for _ in range(copies - 1)]
         self.zs = [z0] * copies if z0 is None else [z0] + [z0.clone() for _ in range(copies - 1)]
-        self.out = torch.empty((self.M, self.N), dtype=torch.float16, device="cuda")
+        self.out = torch.empty((self.M, self.N), dtype=torch.float32 if self.out_f32 else torch.float16,
+                               device="cuda")
         self.ws = w.alloc_workspace(self.M, self.N, self.K, self.G)
         self.i = 0
         self.bytes = alg_bytes(self.M, self.K, self.N, self.G, self.asym)
         self.flops = alg_flops(self.M, self.K, self.N)
 
     pdl = True  # back-to-back steps read weights no step writes: programmatic dependent launch is valid
+    out_f32 = False  # a row shard of a tensor-parallel layer writes fp32 partials
 
     def step(self, stream=None):
         j = self.i % len(self.bs)
         self.i += 1
         self.w.w4a16_gemm(self.a, self.bs[j], self.ss[j], self.zs[j], self.G, self.zp, out=self.out,
-                          workspace=self.ws, stream=stream, pdl=self.pdl)
+                          workspace=self.ws, stream=stream, pdl=self.pdl, out_f32=self.out_f32)
 
     def launches_per_step(self):
         # The library's automatic choice: tensor-core GEMM (one launch per 128 rows) above 32 rows,
@@ -442,8 +444,55 @@ def run_extras(torch, w, peaks):
     p = Problem(w, torch, c, copies_for(alg_bytes(32, 4096, 14336, 128, True)), b=bkn)
     ex["config4_M32"] = summary(p, measure_problem(torch, p, 16, 20), peaks, tensor_bound=True)
     del p
+    # larger batches on the same layer (tensor-core GEMM)
+    for M in (64, 128, 256):
+        cm = synth.make_case(M, 4096, 14336, 128, sym=False, seed=3)
+        p = Problem(w, torch, cm, copies_for(alg_bytes(M, 4096, 14336, 128, True)))
+        ex[f"config4_M{M}"] = summary(p, measure_problem(torch, p, 16, 20), peaks, tensor_bound=True)
+        del p
+    ex.update(run_tp(torch, w, peaks))
     ex.update(run_stack(torch, w, peaks))
     return ex
+
+
+def run_tp(torch, w, peaks):
+    """One rank's share of the decode layer (M=1, K=4096, N=14336, G=128) under P-way tensor
+    parallelism, for P = 2, 4, 8: its column shard (N/P output columns), its row shard (K/P rows,
+    fp32 partial) and the reduction of P partials that closes a row-parallel layer. The
+    collective that brings the partials together is not part of it (one GPU here)."""
+    res = {}
+    c = synth.config2()
+    K, N, G = c["K"], c["N"], c["G"]
+    for P in (2, 4, 8):
+        nc, kr = N // P, K // P
+        col = dict(c, N=nc, b=c["b"][:, :nc // 8], s=c["s"][:, :nc])
+        row = dict(c, K=kr, a=np.ascontiguousarray(c["a"][:, :kr]), b=c["b"][:kr], s=c["s"][:kr // G])
+        pc = Problem(w, torch, col, copies_for(alg_bytes(1, K, nc, G, False)))
+        t_col = measure_problem(torch, pc, 64, 20)
+        del pc
+        Problem.out_f32 = True
+        try:
+            pr = Problem(w, torch, row, copies_for(alg_bytes(1, kr, N, G, False)))
+            t_row = measure_problem(torch, pr, 64, 20)
+        finally:
+            Problem.out_f32 = False
+        del pr
+        parts = [torch.randn((1, N), dtype=torch.float32, device="cuda") for _ in range(P)]
+        red_out = torch.empty((1, N), dtype=torch.float16, device="cuda")
+
+        def red(parts=parts, red_out=red_out):
+            w.w4a16_reduce_partials(parts, out=red_out)
+
+        t_red = measure_problem(torch, type("P", (), {"step": staticmethod(red)})(), 64, 20)
+        roof_col = alg_bytes(1, K, nc, G, False) / (peaks["hbm_gbs"] * 1e9)
+        roof_row = alg_bytes(1, kr, N, G, False) / (peaks["hbm_gbs"] * 1e9)
+        res[f"tp{P}_decode_rank"] = {"col_shard_us": round(t_col * 1e6, 3),
+                                     "col_frac_of_roofline": round(roof_col / t_col, 4),
+                                     "row_shard_us": round(t_row * 1e6, 3),
+                                     "row_frac_of_roofline": round(roof_row / t_row, 4),
+                                     "reduce_us": round(t_red * 1e6, 3),
+                                     "row_plus_reduce_us": round((t_row + t_red) * 1e6, 3)}
+    return res
 
 
 def measure_load_ct(torch, w, peaks):

@@ -190,8 +190,8 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  *     timeout path only.
  *   wait_limit_us: 0 = the default limit (2 s) on every device-side wait,
  *     else that many microseconds.
- *   launch_flags: 0 or W4A16_LAUNCH_PDL. With W4A16_LAUNCH_PDL the mma.sync
- *     GEMV is launched with programmatic dependent launch: it may start while
+ *   launch_flags: 0, or a bit set of W4A16_LAUNCH_PDL and W4A16_OUT_F32.
+ *     With W4A16_LAUNCH_PDL the mma.sync GEMV is launched with programmatic dependent launch: it may start while
  *     the kernel before it on the stream is still running, and streams its
  *     packed weights, scales and zeros right away; it waits for that kernel to
  *     finish (and its writes to be visible) before it reads A or writes out
@@ -199,10 +199,18 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  *     not write b_packed, scales or qzeros (a GEMM after another GEMM or an
  *     activation kernel qualifies; a GEMM right after the w4a16_repack that
  *     produced its weights does not). Other kernels ignore the flag.
+ *     W4A16_OUT_F32 (any kernel): `out` is fp32 [M, N], 4-byte aligned, and
+ *     receives the fp32 sums unrounded instead of their fp16 rounding. This is
+ *     one K-shard's share of a row-parallel (K-split) layer: pass rows
+ *     [k0, k1) of b_packed (k0, k1 multiples of G), rows [k0/G, k1/G) of
+ *     scales and qzeros, and A's columns [k0, k1) as a contiguous
+ *     [M, k1 - k0] array (the layout a column-parallel layer before it leaves
+ *     on each rank), with K = k1 - k0; then add the shards' outputs in a
+ *     fixed order and round once (w4a16_reduce_partials).
  */
 enum { W4A16_KERNEL_AUTO = 0, W4A16_KERNEL_GEMV = 1, W4A16_KERNEL_TC = 2, W4A16_KERNEL_GEMV_FMA = 3 };
 enum { W4A16_DEBUG_STALL_LOADS = 1 };
-enum { W4A16_LAUNCH_PDL = 1 };
+enum { W4A16_LAUNCH_PDL = 1, W4A16_OUT_F32 = 2 };
 typedef struct {
     int32_t kernel;
     int32_t split_k;
@@ -229,6 +237,37 @@ W4A16_API w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const 
  * Errors: INVALID_ARG for NULL pointers; CUDA for a failed copy.
  */
 W4A16_API w4a16_status w4a16_workspace_status(void* workspace, int32_t clear, int32_t* status, void* stream);
+
+/*
+ * w4a16_reduce_partials — out = fp16(parts[0] + parts[1] + ... + parts[P-1]).
+ *
+ * Cited operation: the tensor-parallel layers of section "Arquitectura del
+ * Sistema" of the kerneldigest.dev page on LLM inference with TP, where the
+ * decode step ends each parallel layer with an all-reduce. A row-parallel
+ * (K-split) layer's shards each produce an fp32 partial of the output
+ * (w4a16_gemm_ex with W4A16_OUT_F32); the layer's output is their sum, rounded
+ * once. This call is that sum and rounding, after the partials have been
+ * brought together (an all-gather), or it rounds an all-reduced sum (P = 1).
+ *
+ *   parts  host array of P pointers to fp32 [M, N] device arrays, each 16-byte
+ *          aligned. An array may be another GPU's memory mapped into this
+ *          device's address space (peer access, CUDA IPC); it is read with
+ *          plain loads. The caller orders the writes that produced the parts
+ *          before this call (same stream, events, or a collective's completion).
+ *   P      1..16 (P = 1 only rounds).
+ *   M, N   M >= 1, N >= 8, N % 8 == 0.
+ *   out    fp16 [M, N] device array, 16-byte aligned; fully overwritten; must
+ *          not overlap any part.
+ *   stream cudaStream_t as void*.
+ * Every element is summed in fp32 in index order (((p0 + p1) + p2) + ...) and
+ * rounded to fp16 to nearest even: ranks that reduce the same parts get
+ * bit-identical outputs.
+ * Errors: INVALID_ARG for a NULL pointer, P, M or N outside its range, a
+ * misaligned pointer or an overlap; UNSUPPORTED when the current device is not
+ * sm_100; CUDA for a launch failure.
+ */
+W4A16_API w4a16_status w4a16_reduce_partials(const void* const* parts, int32_t P, int64_t M, int64_t N, void* out,
+                                             void* stream);
 
 /*
  * w4a16_gemm_noalloc — w4a16_gemm for callers that cannot allocate device memory.

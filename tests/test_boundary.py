@@ -127,7 +127,7 @@ def test_options_are_checked():
     o = w.W4A16Options(1, 1025)
     rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
     assert rc == w.W4A16_ERR_INVALID_ARG
-    o = w.W4A16Options(0, 0, 0, 0, 2)   # an undefined launch flag
+    o = w.W4A16Options(0, 0, 0, 0, 4)   # an undefined launch flag
     rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, OUT, None, 0, None, ctypes.byref(o))
     assert rc == w.W4A16_ERR_INVALID_ARG
     assert "launch flag" in w.lib.w4a16_last_error().decode()
@@ -216,3 +216,33 @@ def test_noalloc_checks_on_host():
     assert "GEMV kernels only" in w.lib.w4a16_last_error().decode()
     assert int(w.lib.w4a16_noalloc_scratch_bytes()) == 8 << 20
     del v
+
+
+def test_fp32_output_alignment_is_checked():
+    # W4A16_OUT_F32: the fp32 output needs 4-byte alignment (checked before any device query)
+    o = w.W4A16Options(0, 0, 0, 0, w.OUT_F32)
+    rc = w.lib.w4a16_gemm_ex(GOOD, GOOD2, GOOD3, None, 1, 64, 256, 128, 8, ctypes.c_void_p(OUT.value + 2), None, 0,
+                             None, ctypes.byref(o))
+    assert rc == w.W4A16_ERR_INVALID_ARG
+    assert "fp32 out" in w.lib.w4a16_last_error().decode()
+
+
+@pytest.mark.parametrize("P,M,N,part_off,out_off,why", [
+    (0, 1, 8, 0, 0, "P must be"), (17, 1, 8, 0, 0, "P must be"), (1, 0, 8, 0, 0, "M must be"),
+    (1, 1, 12, 0, 0, "N must be"), (1, 1, 8, 4, 0, "parts must be 16-byte aligned"),
+    (1, 1, 8, 0, 8, "out must be 16-byte aligned"), (1, 1, 8, None, 0, "NULL pointer in parts"),
+])
+def test_reduce_partials_checks_on_host(P, M, N, part_off, out_off, why):
+    base = 1 << 20
+    ptrs = [None if part_off is None else base + 4096 * i + part_off for i in range(max(P, 1))]
+    arr = (ctypes.c_void_p * len(ptrs))(*ptrs)
+    rc = w.lib.w4a16_reduce_partials(arr, P, M, N, ctypes.c_void_p(base + (1 << 16) + out_off), None)
+    assert rc == w.W4A16_ERR_INVALID_ARG
+    assert why in w.lib.w4a16_last_error().decode()
+
+
+def test_reduce_partials_rejects_overlap():
+    base = 1 << 20
+    arr = (ctypes.c_void_p * 2)(base, base + 4096)
+    rc = w.lib.w4a16_reduce_partials(arr, 2, 4, 64, ctypes.c_void_p(base + 4096 + 512), None)
+    assert rc == w.W4A16_ERR_INVALID_ARG and "overlaps" in w.lib.w4a16_last_error().decode()

@@ -32,6 +32,8 @@ class W4A16Options(ctypes.Structure):
 
 DEBUG_STALL_LOADS = 1
 LAUNCH_PDL = 1
+OUT_F32 = 2
+MAX_REDUCE_PARTS = 16
 
 
 _p, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
@@ -61,6 +63,8 @@ lib.w4a16_noalloc_status.argtypes = [_i32, ctypes.POINTER(ctypes.c_int32), _p]
 lib.w4a16_noalloc_status.restype = ctypes.c_int
 lib.w4a16_noalloc_scratch_bytes.argtypes = []
 lib.w4a16_noalloc_scratch_bytes.restype = _sz
+lib.w4a16_reduce_partials.argtypes = [ctypes.POINTER(ctypes.c_void_p), _i32, _i64, _i64, _p, _p]
+lib.w4a16_reduce_partials.restype = ctypes.c_int
 lib.w4a16_status_string.argtypes = [ctypes.c_int]
 lib.w4a16_status_string.restype = ctypes.c_char_p
 lib.w4a16_last_error.argtypes = []
@@ -68,7 +72,8 @@ lib.w4a16_last_error.restype = ctypes.c_char_p
 
 EXPORTED = ("w4a16_repack", "w4a16_load_ct", "w4a16_gemm_kernel_choice", "w4a16_gemm_workspace_bytes", "w4a16_gemm", "w4a16_gemm_ex_workspace_bytes",
             "w4a16_gemm_ex", "w4a16_workspace_status", "w4a16_status_string", "w4a16_last_error",
-            "w4a16_gemm_noalloc", "w4a16_gemm_noalloc_ex", "w4a16_noalloc_status", "w4a16_noalloc_scratch_bytes")
+            "w4a16_gemm_noalloc", "w4a16_gemm_noalloc_ex", "w4a16_noalloc_status", "w4a16_noalloc_scratch_bytes",
+            "w4a16_reduce_partials")
 
 
 class W4A16Error(RuntimeError):
@@ -184,11 +189,12 @@ def w4a16_load_ct(ckpt_nk8: torch.Tensor, scale_ng: torch.Tensor, zero_n8g: torc
 def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qzeros: torch.Tensor | None,
                group_size: int, zp_bias: int = 8, out: torch.Tensor | None = None,
                workspace: torch.Tensor | None = None, stream=None, kernel=None, split_k: int = 0,
-               debug_flags: int = 0, wait_limit_us: int = 0, pdl: bool = False):
+               debug_flags: int = 0, wait_limit_us: int = 0, pdl: bool = False, out_f32: bool = False):
     """out[M, N] = fp16(fp32(a) @ ((q - z) * s)) on the GPU (see include/w4a16.h).
 
     pdl=True sets W4A16_LAUNCH_PDL: only when the kernel before this call on the stream does not
-    write b_packed, scales or qzeros."""
+    write b_packed, scales or qzeros. out_f32=True sets W4A16_OUT_F32: `out` is fp32 and gets the
+    sums unrounded (one K-shard's partial of a row-parallel layer; see w4a16_reduce_partials)."""
     pa = _dev(a, "a", (torch.float16,))
     pb = _dev(b_packed, "b_packed", (torch.int32, torch.uint32))
     ps = _dev(scales, "scales", (torch.float16,))
@@ -203,18 +209,41 @@ def w4a16_gemm(a: torch.Tensor, b_packed: torch.Tensor, scales: torch.Tensor, qz
         raise ValueError("scales must be [K/G, N]")
     if qzeros is not None and tuple(qzeros.shape) != (K // group_size, N // 8):
         raise ValueError("qzeros must be [K/G, N/8]")
+    odt = torch.float32 if out_f32 else torch.float16
     if out is None:
-        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
-    po = _dev(out, "out", (torch.float16,))
+        out = torch.empty((M, N), dtype=odt, device=a.device)
+    po = _dev(out, "out", (odt,))
     if tuple(out.shape) != (M, N):
         raise ValueError("out must be [M, N]")
     if workspace is None:
         workspace = alloc_workspace(M, N, K, group_size, a.device, kernel, split_k)
     pw = _dev(workspace, "workspace", (torch.uint8,))
-    o = _opts(kernel, split_k, debug_flags, wait_limit_us, LAUNCH_PDL if pdl else 0)
+    o = _opts(kernel, split_k, debug_flags, wait_limit_us, (LAUNCH_PDL if pdl else 0) | (OUT_F32 if out_f32 else 0))
     args = (pa, pb, ps, pz, M, N, K, group_size, zp_bias, po, pw, workspace.numel(), _stream_ptr(stream))
     rc = lib.w4a16_gemm(*args) if o is None else lib.w4a16_gemm_ex(*args, o)
     _check(rc, "w4a16_gemm")
+    return out
+
+
+def w4a16_reduce_partials(parts, out: torch.Tensor | None = None, stream=None):
+    """out[M, N] = fp16(parts[0] + parts[1] + ...), summed in fp32 in list order, on the GPU.
+
+    parts: 1..16 fp32 CUDA tensors of one shape [M, N] (N % 8 == 0), each 16-byte aligned."""
+    parts = list(parts)
+    if not 1 <= len(parts) <= MAX_REDUCE_PARTS:
+        raise ValueError(f"between 1 and {MAX_REDUCE_PARTS} parts are needed, got {len(parts)}")
+    ptrs = [_dev(t, f"parts[{i}]", (torch.float32,)).value for i, t in enumerate(parts)]
+    shape = tuple(parts[0].shape)
+    if len(shape) != 2 or any(tuple(t.shape) != shape for t in parts):
+        raise ValueError("parts must be 2-D tensors of one shape")
+    M, N = shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=parts[0].device)
+    po = _dev(out, "out", (torch.float16,))
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be [M, N]")
+    arr = (ctypes.c_void_p * len(ptrs))(*ptrs)
+    _check(lib.w4a16_reduce_partials(arr, len(ptrs), M, N, po, _stream_ptr(stream)), "w4a16_reduce_partials")
     return out
 
 

@@ -17,6 +17,19 @@ namespace w4a16 {
 constexpr size_t kWsHeader = 256;
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Output of a GEMM launch: the layer's fp16 result (rounded to nearest even), or the
+// fp32 sums themselves, unrounded, when the call computes one K-shard's share of a
+// row-parallel layer whose shards are added up later (W4A16_OUT_F32).
+struct OutPtr {
+    __half* h;  // fp16 [M, N], or nullptr
+    float* f;   // fp32 [M, N], or nullptr
+    __device__ __forceinline__ void put(int64_t i, float v) const {
+        if (f) f[i] = v;
+        else h[i] = __float2half_rn(v);
+    }
+    OutPtr rows(int64_t m0, int64_t N) const { return {h ? h + m0 * N : nullptr, f ? f + m0 * N : nullptr}; }
+};
+
 // Device-side wait policy for the pipelined kernels: the limit on each wait,
 // and (tests only) a switch that makes the load issuers issue nothing.
 struct WaitPolicy {
@@ -61,7 +74,7 @@ GemvPlan plan_gemv(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_reque
 bool gemv_mma_supported(int64_t N, int64_t K, const void* a, const void* b, const void* s, const void* z);
 GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_request, int sm_count);
 cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M,
-                            int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace,
+                            int64_t N, int64_t K, int32_t G, int32_t zp_bias, OutPtr out, void* workspace,
                             const GemvPlan& plan, const WaitPolicy& wp, cudaStream_t st);
 
 // Largest rows-per-CTA slab the GEMV stages in shared memory for an explicit split.
@@ -80,7 +93,7 @@ struct TcPlan {
 bool tc_supported(int64_t M, int64_t N, int64_t K, int32_t G, const void* a, const void* b);
 TcPlan plan_tc(int64_t M, int64_t N, int64_t K, int32_t G, int sm_count, int split_k_request);
 cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M, int64_t N,
-                      int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace, const TcPlan& plan,
+                      int64_t K, int32_t G, int32_t zp_bias, OutPtr out, void* workspace, const TcPlan& plan,
                       const WaitPolicy& wp, cudaStream_t st);
 
 cudaError_t launch_repack(const uint32_t* ckpt, uint32_t* out, int64_t N, int64_t K, cudaStream_t st);
@@ -89,7 +102,13 @@ cudaError_t launch_ct_load(const uint32_t* ckpt, const uint16_t* s_ng, const uin
                            uint16_t* s_gn, uint32_t* z_gn8, int64_t N, int64_t K, int64_t ngroups, cudaStream_t st);
 
 cudaError_t launch_gemv(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z,
-                        int64_t M, int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out,
+                        int64_t M, int64_t N, int64_t K, int32_t G, int32_t zp_bias, OutPtr out,
                         void* workspace, const GemvPlan& plan, const WaitPolicy& wp, cudaStream_t st);
+
+// Sum of P fp32 [M, N] partials in fixed order, rounded once to fp16 (16-byte aligned
+// pointers, M * N % 8 == 0).
+constexpr int kMaxReduceParts = 16;
+cudaError_t launch_reduce_partials(const float* const* parts, int P, int64_t M, int64_t N, __half* out, int sm_count,
+                                   cudaStream_t st);
 
 }  // namespace w4a16

@@ -61,7 +61,7 @@ struct GemvArgs {
     const uint32_t* b;    // [K, N/8]
     const __half* s;      // [K/G, N]
     const uint32_t* z;    // [K/G, N/8] or nullptr
-    __half* out;          // [M, N]
+    OutPtr out;           // [M, N]
     float* partials;      // [split][MT][N]
     uint32_t* counters;   // [col_tiles]
     int* status;          // workspace status word (TMA kernel), or nullptr
@@ -240,7 +240,7 @@ __device__ __forceinline__ void finish_cta(const GemvArgs& p, const float2 (&tot
             const int64_t n = n0 + threadIdx.x + q * kThreads;
             if (n < p.N)
 #pragma unroll
-                for (int m = 0; m < MT; ++m) p.out[(int64_t)m * p.N + n] = __float2half_rn(part[m][q]);
+                for (int m = 0; m < MT; ++m) p.out.put((int64_t)m * p.N + n, part[m][q]);
         }
         return;
     }
@@ -268,7 +268,7 @@ __device__ __forceinline__ void finish_cta(const GemvArgs& p, const float2 (&tot
             for (int m = 0; m < MT; ++m) {
                 float acc = 0.f;
                 for (int y = 0; y < p.split; ++y) acc += __ldcg(p.partials + ((int64_t)y * MT + m) * p.N + n);
-                p.out[(int64_t)m * p.N + n] = __float2half_rn(acc);
+                p.out.put((int64_t)m * p.N + n, acc);
             }
         }
     }
@@ -590,7 +590,7 @@ size_t gemv_smem_bytes(int64_t M, int64_t K, int split_k) {
 }
 
 cudaError_t launch_gemv(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z,
-                        int64_t M, int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out,
+                        int64_t M, int64_t N, int64_t K, int32_t G, int32_t zp_bias, OutPtr out,
                         void* workspace, const GemvPlan& pl, const WaitPolicy& wp, cudaStream_t st) {
     CUtensorMap bmap;
     if (pl.tma) {
@@ -608,7 +608,7 @@ cudaError_t launch_gemv(const __half* a, const uint32_t* b, const __half* s, con
         args.b = b;
         args.s = s;
         args.z = z;
-        args.out = out + m0 * N;
+        args.out = out.rows(m0, N);
         args.partials = pl.split_k > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.partials_off) : nullptr;
         args.counters = pl.split_k > 1 ? reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + pl.counters_off) : nullptr;
         args.status = workspace ? static_cast<int*>(workspace) : nullptr;

@@ -105,7 +105,7 @@ __host__ __device__ constexpr size_t sk_smem_bytes(int mt) {
 struct SkArgs {
     const __half* s;      // [K/G, N]
     const uint32_t* z;    // [K/G, N/8] or nullptr
-    __half* out;          // [M, N] (this launch's row block)
+    OutPtr out;           // [M, N] (this launch's row block)
     int* status;
     int64_t N, K;
     int tiles;            // 128-column tiles
@@ -510,7 +510,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) v += tots[w * 4 * NI * 32 + src];
                 if (shared_tile) kp[item] = v;
-                else if (n < p.N) p.out[(int64_t)m * p.N + n] = __float2half_rn(v);
+                else if (n < p.N) p.out.put((int64_t)m * p.N + n, v);
             }
         }
         __syncthreads();  // the totals are free again
@@ -537,7 +537,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
                 if (n >= p.N) continue;
                 float v = 0.f;
                 for (int rr = first; rr <= last; ++rr) v += ld_cluster(src[rr - first] + 4 * item);
-                p.out[(int64_t)m * p.N + n] = __float2half_rn(v);
+                p.out.put((int64_t)m * p.N + n, v);
             }
         }
     }
@@ -699,7 +699,7 @@ GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_r
 }
 
 cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M,
-                            int64_t N, int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace,
+                            int64_t N, int64_t K, int32_t G, int32_t zp_bias, OutPtr out, void* workspace,
                             const GemvPlan& pl, const WaitPolicy& wp, cudaStream_t st) {
     char* ws = static_cast<char*>(workspace);
     int dev = 0, sms = 148;
@@ -734,7 +734,7 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         SkArgs args;
         args.s = s;
         args.z = z;
-        args.out = out + m0 * N;
+        args.out = out.rows(m0, N);
         args.status = workspace ? reinterpret_cast<int*>(ws) : nullptr;
         args.N = N;
         args.K = K;

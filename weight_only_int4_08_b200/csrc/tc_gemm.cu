@@ -107,7 +107,7 @@ struct TcArgs {
     const uint32_t* b;     // [K, N/8]
     const __half* s;       // [K/G, N]
     const uint32_t* z;     // [K/G, N/8] or nullptr
-    __half* out;           // [M, N] (already offset to this row block)
+    OutPtr out;            // [M, N] (already offset to this row block)
     float* partials;       // [split][mblk][N]
     uint32_t* counters;    // [n_tiles]
     int* status;           // workspace status word
@@ -545,7 +545,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             if (p.split == 1) {
 #pragma unroll
                 for (int m = 0; m < MN; ++m)
-                    if (m < p.mblk) p.out[(int64_t)m * p.N + n] = __float2half_rn(tot[m]);
+                    if (m < p.mblk) p.out.put((int64_t)m * p.N + n, tot[m]);
             } else {
 #pragma unroll
                 for (int m = 0; m < MN; ++m)
@@ -562,7 +562,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     for (int m = 0; m < p.mblk; ++m) {
                         float a = 0.f;
                         for (int y = 0; y < p.split; ++y) a += __ldcg(p.partials + ((int64_t)y * p.mblk + m) * p.N + n);
-                        p.out[(int64_t)m * p.N + n] = __float2half_rn(a);
+                        p.out.put((int64_t)m * p.N + n, a);
                     }
                     if (et == 0) p.counters[tile] = 0u;
                 }
@@ -678,7 +678,7 @@ TcPlan plan_tc(int64_t M, int64_t N, int64_t K, int32_t G, int sm_count, int spl
 }
 
 cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const uint32_t* z, int64_t M, int64_t N,
-                      int64_t K, int32_t G, int32_t zp_bias, __half* out, void* workspace, const TcPlan& pl,
+                      int64_t K, int32_t G, int32_t zp_bias, OutPtr out, void* workspace, const TcPlan& pl,
                       const WaitPolicy& wp, cudaStream_t st) {
     // Tensor map over the activations [M, K] fp16: box 64 k x MN rows, 128-byte swizzle;
     // rows past M read as zero.
@@ -704,7 +704,7 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
         args.b = b;
         args.s = s;
         args.z = z;
-        args.out = out + m0 * N;
+        args.out = out.rows(m0, N);
         args.partials = reinterpret_cast<float*>(ws + pl.partials_off);
         args.counters = reinterpret_cast<uint32_t*>(ws + pl.counters_off);
         args.status = reinterpret_cast<int*>(ws);

@@ -281,11 +281,14 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
         return fail_arg("unknown kernel option");
     if (opts && (opts->split_k < 0 || opts->split_k > 1024)) return fail_arg("split_k must be in 0..1024");
     if (opts && (opts->debug_flags & ~(uint32_t)W4A16_DEBUG_STALL_LOADS)) return fail_arg("unknown debug flag");
-    if (opts && (opts->launch_flags & ~(uint32_t)W4A16_LAUNCH_PDL)) return fail_arg("unknown launch flag");
-    if (!aligned(a, 2) || !aligned(scales, 2) || !aligned(out, 2)) return fail_arg("fp16 pointers must be 2-byte aligned");
+    if (opts && (opts->launch_flags & ~(uint32_t)(W4A16_LAUNCH_PDL | W4A16_OUT_F32)))
+        return fail_arg("unknown launch flag");
+    const bool out_f32 = opts && (opts->launch_flags & W4A16_OUT_F32);
+    if (!aligned(a, 2) || !aligned(scales, 2)) return fail_arg("fp16 pointers must be 2-byte aligned");
+    if (!aligned(out, out_f32 ? 4 : 2)) return fail_arg(out_f32 ? "fp32 out must be 4-byte aligned" : "fp16 pointers must be 2-byte aligned");
     if (!aligned(b_packed, 4) || (qzeros && !aligned(qzeros, 4))) return fail_arg("int32 pointers must be 4-byte aligned");
     const size_t a_bytes = (size_t)M * K * 2, b_bytes = (size_t)K * N / 2, s_bytes = (size_t)(K / group_size) * N * 2;
-    const size_t z_bytes = qzeros ? (size_t)(K / group_size) * N / 2 : 0, o_bytes = (size_t)M * N * 2;
+    const size_t z_bytes = qzeros ? (size_t)(K / group_size) * N / 2 : 0, o_bytes = (size_t)M * N * (out_f32 ? 4 : 2);
     if (overlaps(out, o_bytes, a, a_bytes) || overlaps(out, o_bytes, b_packed, b_bytes) ||
         overlaps(out, o_bytes, scales, s_bytes) || overlaps(out, o_bytes, qzeros, z_bytes))
         return fail_arg("out overlaps an input");
@@ -320,22 +323,23 @@ w4a16_status w4a16_gemm_ex(const void* a, const void* b_packed, const void* scal
     wp.limit_ns = (opts && opts->wait_limit_us) ? (uint64_t)opts->wait_limit_us * 1000ull : 2000000000ull;
     wp.stall_loads = (opts && (opts->debug_flags & W4A16_DEBUG_STALL_LOADS)) ? 1 : 0;
     wp.pdl = (opts && (opts->launch_flags & W4A16_LAUNCH_PDL)) ? 1 : 0;
+    OutPtr o{out_f32 ? nullptr : static_cast<__half*>(out), out_f32 ? static_cast<float*>(out) : nullptr};
     if (c.kernel == W4A16_KERNEL_TC) {
         e = launch_tc(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
                       static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K, group_size,
-                      zp_bias, static_cast<__half*>(out), workspace, c.tc, wp, st);
+                      zp_bias, o, workspace, c.tc, wp, st);
         return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
     }
     if (c.gemv.mma) {
         e = launch_gemv_mma(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
                             static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K,
-                            group_size, zp_bias, static_cast<__half*>(out), workspace, c.gemv, wp, st);
+                            group_size, zp_bias, o, workspace, c.gemv, wp, st);
         return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
     }
     if (gemv_smem_bytes(M, K, c.gemv.split_k) > 160 * 1024) return fail_arg("split_k too small for this K");
     e = launch_gemv(static_cast<const __half*>(a), static_cast<const uint32_t*>(b_packed),
                     static_cast<const __half*>(scales), static_cast<const uint32_t*>(qzeros), M, N, K,
-                    group_size, zp_bias, static_cast<__half*>(out), workspace, c.gemv, wp, st);
+                    group_size, zp_bias, o, workspace, c.gemv, wp, st);
     return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
 }
 
@@ -344,6 +348,33 @@ w4a16_status w4a16_gemm(const void* a, const void* b_packed, const void* scales,
                         void* out, void* workspace, size_t workspace_bytes, void* stream) {
     return w4a16_gemm_ex(a, b_packed, scales, qzeros, M, N, K, group_size, zp_bias, out, workspace,
                          workspace_bytes, stream, nullptr);
+}
+
+w4a16_status w4a16_reduce_partials(const void* const* parts, int32_t P, int64_t M, int64_t N, void* out,
+                                   void* stream) {
+    g_last_error[0] = 0;
+    if (!parts || !out) return fail_arg("NULL pointer");
+    if (P < 1 || P > kMaxReduceParts) return fail_arg("P must be in 1..16");
+    if (M < 1 || M >= kMaxDim) return fail_arg("M must be in 1..2^31-1");
+    if (N < 8 || N % 8 || N >= kMaxDim) return fail_arg("N must be a positive multiple of 8");
+    if (!aligned(out, 16)) return fail_arg("out must be 16-byte aligned");
+    const size_t pb = (size_t)M * N * 4, ob = (size_t)M * N * 2;
+    const float* fp[kMaxReduceParts];
+    for (int r = 0; r < P; ++r) {
+        if (!parts[r]) return fail_arg("NULL pointer in parts");
+        if (!aligned(parts[r], 16)) return fail_arg("parts must be 16-byte aligned");
+        if (overlaps(out, ob, parts[r], pb)) return fail_arg("out overlaps a part");
+        fp[r] = static_cast<const float*>(parts[r]);
+    }
+    int sms = 0, maj = 0;
+    cudaError_t e = device_info(&sms, &maj);
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (maj != 10) {
+        set_error("unsupported: %s", "this library is built for sm_100 (B200) devices");
+        return W4A16_ERR_UNSUPPORTED;
+    }
+    e = launch_reduce_partials(fp, P, M, N, static_cast<__half*>(out), sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? W4A16_OK : fail_cuda(e);
 }
 
 w4a16_status w4a16_workspace_status(void* workspace, int32_t clear, int32_t* status, void* stream) {
