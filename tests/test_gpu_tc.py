@@ -44,6 +44,19 @@ def test_tc_row_blocks(w, M):
     assert_close(run(w, c, kernel=w.KERNEL_TC), ref(c), f"TC M={M}")
 
 
+@pytest.mark.parametrize("M", [64, 128, 256])
+def test_tc_batch_layer_large_batches(w, M):
+    """The batch-32 layer's shape (K=4096, N=14336, G=128, asymmetric) at 64, 128 and 256 rows,
+    as the bench times it: every row against the oracle on sampled columns (one in each
+    128-column tile, plus the first and the last column), which it computes one by one."""
+    K, N = 4096, 14336
+    c = synth.make_case(M, K, N, 128, sym=False, seed=3)
+    g = np.random.default_rng(M)
+    cols = np.unique(np.concatenate([np.arange(0, N, 128) + g.integers(0, 128, N // 128), [0, N - 1]]))
+    out = run(w, c, kernel=w.KERNEL_TC).cpu().numpy()
+    assert_close(out[:, cols], ref(c, cols=cols), f"TC M={M}")
+
+
 @pytest.mark.parametrize("G", [16, 32, 64, 128, 256])
 @pytest.mark.parametrize("split", [1, 3])
 def test_tc_group_sizes_and_splits(w, G, split):
