@@ -112,6 +112,7 @@ struct SkArgs {
     int tiles_per_cluster;
     int G, zp_bias, nblk, stall_loads;
     uint32_t magic;       // kMagic, passed at run time so that the and-or unpack compiles to one LOP3
+    int shares_mask;      // bit 0: a full cluster splits a tile between CTAs; bit 1: the last, shorter one does
     uint64_t wait_ns;
 };
 
@@ -346,8 +347,17 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         const bool z_ok = p.z && lane < kTileWords && tile * kTileWords + lane < nw;
 
         float acc[4][NT][8];
+        // The fragment's scaled group sums: in registers up to 8 rows (4 NI values per lane, stored to
+        // shared memory once at the fragment's end), in shared memory above, where registers run out.
+        // Measured on B200 (decode GEMV, per-warp timeline): 16 load-FMA-store steps on shared memory
+        // took ~0.24 us per group.
+        constexpr bool kRegTot = MT <= 8;
+        float treg[kRegTot ? 4 * NI : 1];
 #pragma unroll
-        for (int k = 0; k < 4 * NI; ++k) tmine[32 * k] = 0.f;
+        for (int k = 0; k < 4 * NI; ++k) {
+            if constexpr (kRegTot) treg[k] = 0.f;
+            else tmine[32 * k] = 0.f;
+        }
 
         // Copy group gg's scales and zero words of this tile into group buffer gg & 1, one group
         // ahead of use. Chunks past N get zero scales.
@@ -376,8 +386,13 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         if (MT > 1 || (i & 1) == 0) {
-                            float* tp = tmine + 32 * (c * NI + nt * NB + (MT > 1 ? i : i / 2));
-                            *tp = fmaf(sj[i >> 1], acc[c][nt][i], *tp);
+                            const int k = c * NI + nt * NB + (MT > 1 ? i : i / 2);
+                            if constexpr (kRegTot) {
+                                treg[k] = fmaf(sj[i >> 1], acc[c][nt][i], treg[k]);
+                            } else {
+                                float* tp = tmine + 32 * k;
+                                *tp = fmaf(sj[i >> 1], acc[c][nt][i], *tp);
+                            }
                         }
             }
         };
@@ -493,6 +508,10 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         // ---- reduce fragment f over the warps (warp order) ----
         // A tile held by this CTA alone is written out now; the first and the last fragment may be
         // shared with other CTAs of the cluster and are kept (keep[0], keep[1]) for the exchange.
+        if constexpr (kRegTot) {
+#pragma unroll
+            for (int k = 0; k < 4 * NI; ++k) tmine[32 * k] = treg[k];
+        }
         __syncthreads();
         // s_abort is read by every thread between two barriers with no wait in between: uniform.
         if (s_abort == 0) {
@@ -518,8 +537,15 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 
     // ---- tiles shared within the cluster: the first CTA touching a tile sums every part, in rank
     // order, from the CTAs' shared memory (distributed shared memory), then writes the tile ----
-    cluster_sync();
-    if (s_abort == 0) {
+    // Only a cluster whose rank boundaries cut through a tile has shared tiles; the others (every CTA
+    // runs whole tiles) neither read each other's shared memory nor wait for each other. Every CTA
+    // of a cluster computes the same answer, so all of them or none take the cluster barriers.
+    // Measured on B200 (decode GEMV, clusters of 3 CTAs over 3 tiles): the two barriers cost a CTA
+    // ~1.6 us at the end of the launch.
+    const bool cluster_shares =
+        (tile_hi - tile_lo == p.tiles_per_cluster ? p.shares_mask & 1 : p.shares_mask & 2) != 0;
+    if (cluster_shares) cluster_sync();
+    if (cluster_shares && s_abort == 0) {
 #pragma unroll
         for (int d = 0; d < 2; ++d) {
             if (d >= nfrag || (d == 1 && nfrag == 1)) continue;
@@ -541,7 +567,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             }
         }
     }
-    cluster_sync();   // no CTA leaves while another still reads its shared memory
+    if (cluster_shares) cluster_sync();   // no CTA leaves while another still reads its shared memory
 
     // A wait gave up: let the copies already issued land before the CTA's shared memory goes away.
     cp_async_wait_all();
@@ -744,6 +770,19 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         args.zp_bias = zp_bias;
         args.nblk = (int)l.nblk;
         args.magic = kMagic;
+        {
+            // A cluster of S CTAs over `tiles` whole tiles splits a tile between CTAs when a rank
+            // boundary of its units falls inside one.
+            const int64_t T = pl.col_tiles, k = l.cluster_tiles;
+            auto shares = [&](int64_t tiles) {
+                const int64_t U = tiles * l.nblk;
+                for (int r = 1; r < l.cluster; ++r)
+                    if ((U * r / l.cluster) % l.nblk != 0) return true;
+                return false;
+            };
+            const int64_t last_tiles = T - (T - 1) / k * k;
+            args.shares_mask = (shares(k) ? 1 : 0) | (shares(last_tiles) ? 2 : 0);
+        }
         args.stall_loads = wp.stall_loads;
         args.wait_ns = wp.limit_ns;
         const size_t smem = sk_smem_bytes(mt);
