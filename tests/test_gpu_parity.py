@@ -127,6 +127,9 @@ def test_config5_stack_sampled(w, M):
     (15, 256, 136, 16, False),
     (33, 1024, 776, 128, False),
     (1, 4096, 4104, 128, False),  # 4104 = 16*256 + 8: one-word tail tile
+    (5, 1024, 19968, 128, False),  # 156 column tiles, more than the SMs: the 4-warp GEMV
+    (8, 512, 38912, 64, True),     # 304 tiles, G below the unit rows, 4-warp GEMV
+    (1, 256, 19200, 128, True),    # 150 tiles: one tile per CTA, ragged last wave
 ])
 def test_odd_shapes(w, M, K, N, G, sym):
     c = synth.make_case(M, K, N, G, sym=sym, seed=M + K + N)

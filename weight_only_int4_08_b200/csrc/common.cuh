@@ -47,6 +47,7 @@ struct GemvPlan {
     int col_tiles;    // column tiles
     int cluster;      // mma GEMV: CTAs per thread-block cluster
     int cluster_tiles;  // mma GEMV: whole column tiles per cluster
+    int warps;        // mma GEMV: warps per CTA
     int split_k_request;  // the caller's split_k option (0 = automatic)
     size_t ws_bytes;  // workspace bytes needed (0 when split_k == 1)
     size_t counters_off, partials_off;

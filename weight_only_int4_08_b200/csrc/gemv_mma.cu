@@ -54,8 +54,13 @@ namespace {
 #ifndef W4A16_SK_WARPS
 #define W4A16_SK_WARPS 8
 #endif
-constexpr int kWarps = W4A16_SK_WARPS;
-constexpr int kThreads = 32 * kWarps;
+// Warps per CTA: 8 (one CTA per SM), or 4 (two CTAs per SM) for launches of up to 8 rows on
+// layers with more 128-column tiles than the GPU has SMs. Measured on B200 at M=1 (CUDA graphs,
+// programmatic dependent launch, weights larger than L2): K=4096, N=28672 (224 tiles) 23.0 ->
+// 16.4 us with 4 warps; K=4096, N=14336 (112 tiles) 9.96 against 11.37 us, and every narrower
+// layer measured, stay faster with 8.
+constexpr int kWarpsMax = W4A16_SK_WARPS;
+constexpr int kWarpsWide = 4;
 constexpr int kTileN = 128;
 constexpr int kTileWords = kTileN / 8;            // 16 packed words = 64 B per row
 #ifndef W4A16_SK_ROWS
@@ -97,9 +102,9 @@ __host__ __device__ constexpr int tot_per_tile(int mt) { return mt > 1 ? 8 : 4; 
 __host__ __device__ constexpr int tot_per_chunk(int mt) { return tot_per_tile(mt) * n_tiles(mt); }
 // Dynamic shared memory: weight ring, activation ring, fp32 totals, group buffers, and the
 // warp-reduced sums of the (at most two) fragments shared with other CTAs.
-__host__ __device__ constexpr size_t sk_smem_bytes(int mt) {
-    return (size_t)kWarps * kRing * (wstage_bytes(mt) + a_slot_bytes(mt)) +
-           (size_t)kWarps * 4 * tot_per_chunk(mt) * 32 * 4 + (size_t)kWarps * 2 * kGrpBytes + 2 * (size_t)mt * kTileN * 4;
+__host__ __device__ constexpr size_t sk_smem_bytes(int warps, int mt) {
+    return (size_t)warps * kRing * (wstage_bytes(mt) + a_slot_bytes(mt)) +
+           (size_t)warps * 4 * tot_per_chunk(mt) * 32 * 4 + (size_t)warps * 2 * kGrpBytes + 2 * (size_t)mt * kTileN * 4;
 }
 
 struct SkArgs {
@@ -198,9 +203,10 @@ __device__ __forceinline__ float ld_cluster(uint32_t addr) {
 #endif
 // FAST: the group size is a multiple of the unit (kRows), so a group starts only at a unit start
 // (and K is a multiple of kRows); otherwise groups are tracked per 16-row step.
-template <int MT, bool FAST>
-__global__ void __launch_bounds__(kThreads, W4A16_SK_MIN_CTAS)
+template <int kWarps, int MT, bool FAST>
+__global__ void __launch_bounds__(32 * kWarps, W4A16_SK_MIN_CTAS)
 gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ CUtensorMap amap, SkArgs p) {
+    constexpr int kThreads = 32 * kWarps;
     constexpr int kRows = rows_for(MT);            // rows per unit / stage
     constexpr int kSteps = kRows / 16;             // 16-row MMA steps per stage
     constexpr int kWStage = wstage_bytes(MT);
@@ -582,66 +588,78 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 
 using SkFn = void (*)(CUtensorMap, CUtensorMap, SkArgs);
 
-template <bool FAST>
+template <int W, bool FAST>
 SkFn select_sk_t(int mt) {
     switch (mt) {
-        case 1: return gemv_sk_kernel<1, FAST>;
-        case 2: return gemv_sk_kernel<2, FAST>;
-        case 3: return gemv_sk_kernel<3, FAST>;
-        case 4: return gemv_sk_kernel<4, FAST>;
-        case 5: return gemv_sk_kernel<5, FAST>;
-        case 6: return gemv_sk_kernel<6, FAST>;
-        case 7: return gemv_sk_kernel<7, FAST>;
-        case 8: return gemv_sk_kernel<8, FAST>;
-        case 9: return gemv_sk_kernel<9, FAST>;
-        case 10: return gemv_sk_kernel<10, FAST>;
-        case 11: return gemv_sk_kernel<11, FAST>;
-        case 12: return gemv_sk_kernel<12, FAST>;
-        case 13: return gemv_sk_kernel<13, FAST>;
-        case 14: return gemv_sk_kernel<14, FAST>;
-        case 15: return gemv_sk_kernel<15, FAST>;
-        default: return gemv_sk_kernel<16, FAST>;
+        case 1: return gemv_sk_kernel<W, 1, FAST>;
+        case 2: return gemv_sk_kernel<W, 2, FAST>;
+        case 3: return gemv_sk_kernel<W, 3, FAST>;
+        case 4: return gemv_sk_kernel<W, 4, FAST>;
+        case 5: return gemv_sk_kernel<W, 5, FAST>;
+        case 6: return gemv_sk_kernel<W, 6, FAST>;
+        case 7: return gemv_sk_kernel<W, 7, FAST>;
+        case 8: return gemv_sk_kernel<W, 8, FAST>;
+        default: break;
     }
+    if constexpr (W == kWarpsMax) {
+        switch (mt) {
+            case 9: return gemv_sk_kernel<W, 9, FAST>;
+            case 10: return gemv_sk_kernel<W, 10, FAST>;
+            case 11: return gemv_sk_kernel<W, 11, FAST>;
+            case 12: return gemv_sk_kernel<W, 12, FAST>;
+            case 13: return gemv_sk_kernel<W, 13, FAST>;
+            case 14: return gemv_sk_kernel<W, 14, FAST>;
+            case 15: return gemv_sk_kernel<W, 15, FAST>;
+            default: return gemv_sk_kernel<W, 16, FAST>;
+        }
+    }
+    return nullptr;   // 4-warp CTAs serve launches of up to 8 rows only
 }
 // Occupancy queries use the FAST instance (both have the same shared memory and launch bounds).
-SkFn select_sk(int mt, bool fast = true) { return fast ? select_sk_t<true>(mt) : select_sk_t<false>(mt); }
+SkFn select_sk(int warps, int mt, bool fast = true) {
+    if (warps == kWarpsWide && kWarpsWide != kWarpsMax)
+        return fast ? select_sk_t<kWarpsWide, true>(mt) : select_sk_t<kWarpsWide, false>(mt);
+    return fast ? select_sk_t<kWarpsMax, true>(mt) : select_sk_t<kWarpsMax, false>(mt);
+}
+// Index of a warp count in the per-configuration caches below.
+int wix(int warps) { return warps == kWarpsMax ? 0 : 1; }
 
-std::atomic<int> g_sk_occ[kMaxMT + 1];
+std::atomic<int> g_sk_occ[2][kMaxMT + 1];
 
 // Resident CTAs per SM from the kernel's registers and shared memory.
-int sk_ctas_per_sm(int mt) {
-    int n = g_sk_occ[mt].load(std::memory_order_relaxed);
+int sk_ctas_per_sm(int warps, int mt) {
+    int n = g_sk_occ[wix(warps)][mt].load(std::memory_order_relaxed);
     if (n > 0) return n;
     cudaFuncAttributes fa{};
     int regs = 255;
     size_t static_smem = 1024;
-    if (cudaFuncGetAttributes(&fa, select_sk(mt)) == cudaSuccess && fa.numRegs > 0) {
+    if (cudaFuncGetAttributes(&fa, select_sk(warps, mt)) == cudaSuccess && fa.numRegs > 0) {
         regs = fa.numRegs;
         static_smem = fa.sharedSizeBytes;
     }
-    const size_t smem = sk_smem_bytes(mt) + static_smem + 1024;   // + the per-CTA reservation
+    const size_t smem = sk_smem_bytes(warps, mt) + static_smem + 1024;   // + the per-CTA reservation
     const int by_smem = (int)((228 * 1024) / smem);
-    const int by_regs = 65536 / (((regs + 7) / 8 * 8) * kThreads);
+    const int by_regs = 65536 / (((regs + 7) / 8 * 8) * 32 * warps);
     n = std::max(1, std::min(by_smem, by_regs));
-    g_sk_occ[mt].store(n, std::memory_order_relaxed);
+    g_sk_occ[wix(warps)][mt].store(n, std::memory_order_relaxed);
     return n;
 }
 
-std::atomic<int> g_sk_clusters[kMaxMT + 1][kMaxCluster + 1];
+std::atomic<int> g_sk_clusters[2][kMaxMT + 1][kMaxCluster + 1];
 
 // Clusters of S CTAs that can be resident at once (clusters are placed within one GPC each, so
 // this can be less than the resident CTAs divided by S).
-int sk_max_clusters(int mt, int S) {
-    int n = g_sk_clusters[mt][S].load(std::memory_order_relaxed);
+int sk_max_clusters(int warps, int mt, int S) {
+    int n = g_sk_clusters[wix(warps)][mt][S].load(std::memory_order_relaxed);
     if (n > 0) return n;
-    SkFn k = select_sk(mt);
-    const size_t smem = sk_smem_bytes(mt);
+    SkFn k = select_sk(warps, mt);
+    const size_t smem = sk_smem_bytes(warps, mt);
     n = 0;
     if (kMaxCluster > 8) cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3((unsigned)S);
-        cfg.blockDim = dim3(kThreads);
+        cfg.blockDim = dim3(32 * warps);
         cfg.dynamicSmemBytes = smem;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -654,7 +672,7 @@ int sk_max_clusters(int mt, int S) {
     }
     cudaGetLastError();  // a failed query must not leak into the next launch check
     if (n <= 0) n = 1;
-    g_sk_clusters[mt][S].store(n, std::memory_order_relaxed);
+    g_sk_clusters[wix(warps)][mt][S].store(n, std::memory_order_relaxed);
     return n;
 }
 
@@ -662,19 +680,24 @@ int sk_max_clusters(int mt, int S) {
 // all resident at once; the fewest units per CTA wins, then the most CTAs. An explicit split asks
 // for that many CTAs per tile (at most a cluster, at most one per unit).
 struct SkLayout {
-    int cluster, cluster_tiles, ctas;
+    int cluster, cluster_tiles, ctas, warps;
     int64_t nblk;
 };
+int sk_warps(int mt, int64_t N, int sm_count) {
+    const int64_t T = (N + kTileN - 1) / kTileN;
+    return mt <= 8 && T > sm_count ? kWarpsWide : kWarpsMax;
+}
 SkLayout sk_layout(int mt, int64_t N, int64_t K, int split_k_request, int sm_count) {
     const int64_t T = (N + kTileN - 1) / kTileN, nblk = (K + rows_for(mt) - 1) / rows_for(mt);
+    const int warps = sk_warps(mt, N, sm_count);
     int best_s = 1, best_k = 1;
     if (split_k_request > 0) {
         best_s = (int)std::min<int64_t>(std::min(split_k_request, kMaxCluster), nblk);
     } else {
-        const int64_t slots = (int64_t)std::max(sm_count, 1) * sk_ctas_per_sm(mt);
+        const int64_t slots = (int64_t)std::max(sm_count, 1) * sk_ctas_per_sm(warps, mt);
         int64_t best_cost = INT64_MAX, best_ctas = 0;
         for (int S = 1; S <= kMaxCluster; ++S) {
-            const int64_t qmax = std::min<int64_t>({T, slots / S, (int64_t)sk_max_clusters(mt, S)});
+            const int64_t qmax = std::min<int64_t>({T, slots / S, (int64_t)sk_max_clusters(warps, mt, S)});
             for (int64_t Q = 1; Q <= qmax; ++Q) {
                 const int64_t k = (T + Q - 1) / Q;
                 if ((Q - 1) * k >= T) continue;   // the same k with fewer clusters
@@ -694,6 +717,7 @@ SkLayout sk_layout(int mt, int64_t N, int64_t K, int split_k_request, int sm_cou
     l.cluster = best_s;
     l.cluster_tiles = best_k;
     l.ctas = (int)((T + best_k - 1) / best_k) * best_s;
+    l.warps = warps;
     l.nblk = nblk;
     return l;
 }
@@ -718,6 +742,7 @@ GemvPlan plan_gemv_mma(int64_t M, int64_t N, int64_t K, int32_t G, int split_k_r
     const SkLayout l = sk_layout(pl.m_rows, N, K, split_k_request, sm_count);
     pl.cluster = l.cluster;
     pl.cluster_tiles = l.cluster_tiles;
+    pl.warps = l.warps;
     pl.split_k = l.ctas;
     pl.split_k_request = split_k_request;
     pl.ws_bytes = 0;  // partial sums stay in the clusters' shared memory
@@ -735,7 +760,7 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         const int mt = (int)std::min<int64_t>(kMaxMT, M - m0);
         const int rows = rows_for(mt);
         // Row blocks of another size than the first take their own layout (stage rows differ).
-        const SkLayout l = mt == pl.m_rows ? SkLayout{pl.cluster, pl.cluster_tiles, pl.split_k, (K + rows - 1) / rows}
+        const SkLayout l = mt == pl.m_rows ? SkLayout{pl.cluster, pl.cluster_tiles, pl.split_k, pl.warps, (K + rows - 1) / rows}
                                            : sk_layout(mt, N, K, split_req, sms);
         CUtensorMap bmap, amap;
         {
@@ -785,8 +810,8 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         }
         args.stall_loads = wp.stall_loads;
         args.wait_ns = wp.limit_ns;
-        const size_t smem = sk_smem_bytes(mt);
-        SkFn k = select_sk(mt, G % rows == 0);
+        const size_t smem = sk_smem_bytes(l.warps, mt);
+        SkFn k = select_sk(l.warps, mt, G % rows == 0);
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         if (l.cluster > 8) {
@@ -795,7 +820,7 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         }
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3((unsigned)l.ctas);
-        cfg.blockDim = dim3(kThreads);
+        cfg.blockDim = dim3(32 * l.warps);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
         cudaLaunchAttribute attr[2];
