@@ -364,7 +364,7 @@ def run_gpu(args):
     Problem.pdl = args.pdl
     achieved = prob.bytes / per_launch / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
-    kernel_name = "tc_gemm_kernel<32, true>" if args.workload == "batch32" else "gemv_sk_kernel<1, true>"
+    kernel_name = "tc_gemm_kernel<32, true>" if args.workload == "batch32" else "gemv_sk_kernel<8, 1, true>"
     traffic = traffic_from_profiles("tc_m32_k4096_n14336" if args.workload == "batch32" else "gemv_m1_k4096_n14336")
     if traffic is not None:  # per step, like `achieved`
         traffic = traffic * prob.launches_per_step()
