@@ -191,14 +191,15 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  *   wait_limit_us: 0 = the default limit (2 s) on every device-side wait,
  *     else that many microseconds.
  *   launch_flags: 0, or a bit set of W4A16_LAUNCH_PDL and W4A16_OUT_F32.
- *     With W4A16_LAUNCH_PDL the mma.sync GEMV is launched with programmatic dependent launch: it may start while
+ *     With W4A16_LAUNCH_PDL the mma.sync GEMV and the tensor-core GEMM are
+ *     launched with programmatic dependent launch: a kernel may start while
  *     the kernel before it on the stream is still running, and streams its
  *     packed weights, scales and zeros right away; it waits for that kernel to
  *     finish (and its writes to be visible) before it reads A or writes out
  *     or the workspace. The caller guarantees that the preceding kernel does
  *     not write b_packed, scales or qzeros (a GEMM after another GEMM or an
  *     activation kernel qualifies; a GEMM right after the w4a16_repack that
- *     produced its weights does not). Other kernels ignore the flag.
+ *     produced its weights does not). The CUDA-core GEMV ignores the flag.
  *     W4A16_OUT_F32 (any kernel): `out` is fp32 [M, N], 4-byte aligned, and
  *     receives the fp32 sums unrounded instead of their fp16 rounding. This is
  *     one K-shard's share of a row-parallel (K-split) layer: pass rows

@@ -1,6 +1,7 @@
 """Programmatic dependent launch (W4A16_LAUNCH_PDL) keeps every dependency.
 
-With the flag, a GEMV may start while the kernel before it is still running and
+With the flag, a GEMV or a tensor-core GEMM (48 and 200 rows: one and two row-block
+launches) may start while the kernel before it is still running and
 stream its weights early, but it must read its activations only after that
 kernel has finished. A chain of layers where each call's input is the previous
 call's output makes the dependency real: the chained outputs with the flag must
@@ -44,10 +45,11 @@ def _chain(w, x0, layers, G, pdl, outs):
     return outs
 
 
-@pytest.mark.parametrize("M,sym", [(1, True), (4, False)])
+@pytest.mark.parametrize("M,sym", [(1, True), (4, False), (48, False), (200, True)])
 def test_pdl_chain_matches_plain_chain(w, M, sym):
     K, G, n = 2048, 128, 6
     layers = _layers(n, K, G, sym, seed=40 + M)
+    assert (w.w4a16_gemm_kernel_choice(M, K, K, G) == w.KERNEL_TC) == (M > 32)
     x0 = dev(synth.fp16_normal(np.random.default_rng(7), (M, K)))
     plain = _chain(w, x0, layers, G, False, [torch.empty((M, K), dtype=torch.float16, device="cuda") for _ in layers])
     fast = _chain(w, x0, layers, G, True, [torch.empty((M, K), dtype=torch.float16, device="cuda") for _ in layers])
@@ -59,9 +61,12 @@ def test_pdl_chain_matches_plain_chain(w, M, sym):
     assert_close(plain[0], ref, "first layer vs oracle")
 
 
-def test_pdl_chain_in_a_cuda_graph(w):
-    K, G, n, M = 2048, 128, 6, 1
+@pytest.mark.parametrize("M", [1, 48])
+def test_pdl_chain_in_a_cuda_graph(w, M):
+    K, G, n = 2048, 128, 6
     layers = _layers(n, K, G, True, seed=60)
+    if M > 32:
+        assert w.w4a16_gemm_kernel_choice(M, K, K, G) == w.KERNEL_TC
     x0 = dev(synth.fp16_normal(np.random.default_rng(8), (M, K)))
     plain = _chain(w, x0, layers, G, False, [torch.empty((M, K), dtype=torch.float16, device="cuda") for _ in layers])
     outs = [torch.empty((M, K), dtype=torch.float16, device="cuda") for _ in layers]

@@ -208,6 +208,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = s_tmem;
+    // With programmatic dependent launch the next kernel on the stream may be scheduled now. This
+    // one waits for the kernel before it (griddepcontrol.wait) only where it reads what that kernel
+    // may have written (the activations) and before it writes (output, workspace); the weights,
+    // scales and zeros stream from the start. Without the launch attribute both are no-ops.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == kAProducer) {
         // ------------------------------------------------- activation producer
@@ -215,6 +220,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         // 128-byte swizzle, rows past M read as zero). Converged loop, one elected lane issuing.
         const bool leader = ptx::elect_one();
         if (leader) ptx::prefetch_tensormap(&amap);
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // the activations come from the kernel before
         int issued = 0;
         for (int i = 0; i < nst && !p.stall_loads; ++i) {
             const int s = i % AS;
@@ -541,6 +547,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         // One decision for all 128 epilogue threads (a timeout seen by any of them,
         // or by another role, skips the output), so the named barriers below match.
         const bool bad = ptx::named_bar_or(1, 128, !ok || s_abort);
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // before the first write
         if (!bad) {
             if (p.split == 1) {
 #pragma unroll
@@ -572,7 +579,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (s_abort && threadIdx.x == 0 && p.status) atomicExch(p.status, (int)W4A16_ERR_TIMEOUT);
+    if (s_abort && threadIdx.x == 0 && p.status) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        atomicExch(p.status, (int)W4A16_ERR_TIMEOUT);
+    }
     if (warp == kMmaWarp) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, C::kTmemCols);
@@ -724,8 +734,19 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
         const size_t smem = tc_launch_smem(pl.mn);
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        k<<<dim3((unsigned)pl.n_tiles, (unsigned)pl.split_k), tc_threads(pl.mn), smem, st>>>(amap, wmap, args);
-        e = cudaGetLastError();
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)pl.n_tiles, (unsigned)pl.split_k);
+        cfg.blockDim = dim3(tc_threads(pl.mn));
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        // Later row blocks of one call read the same weights and write other rows: they may overlap
+        // the block before them whenever the call may overlap its predecessor.
+        cfg.numAttrs = wp.pdl ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, k, amap, wmap, args);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
