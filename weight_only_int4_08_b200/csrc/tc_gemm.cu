@@ -507,19 +507,26 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         int64_t g_idx = seg.k_lo / p.G;                    // group of the current segment
         int64_t bound = (g_idx + 1) * p.G;                 // its end row (or the slab end)
         const int64_t g_last = (seg.k_hi - 1) / p.G;       // last group of the slab
-        // Segments are consecutive groups; their scales are loaded four segments ahead in a
-        // register ring (a DRAM round trip is longer than one segment).
-        auto scale_of = [&](int64_t g) -> float {
-            return g <= g_last ? fscale * __half2float(p.s[g * p.N + n]) : 0.f;
+        // Segments are consecutive groups. Their scales are loaded eight segments ahead into a ring
+        // of raw fp16 bits and converted only when their segment is read. Converting at load time
+        // made the thread wait for every load at once: a per-stage timeline on B200 (M = 32) showed
+        // this epilogue as the slowest role, ~0.4-0.55 us per segment for 0.06 us of work, behind
+        // scale loads that queue with the weight stream in DRAM for 1-4 us.
+        constexpr int kSR = 8;
+        auto scale_raw = [&](int64_t g) -> unsigned short {
+            return g <= g_last ? __ldg(reinterpret_cast<const unsigned short*>(p.s) + g * p.N + n)
+                               : (unsigned short)0;
         };
+        unsigned short sr[kSR];
+#pragma unroll
+        for (int j = 0; j < kSR; ++j) sr[j] = scale_raw(g_idx + j);
         int64_t k_end = min(seg.k_hi, bound) - 16;
-        float sc = scale_of(g_idx), sc1 = scale_of(g_idx + 1), sc2 = scale_of(g_idx + 2), sc3 = scale_of(g_idx + 3);
         while (k_end >= seg.k_lo && ok) {
             const int64_t k_next = k_end + 16 < seg.k_hi ? min(seg.k_hi, bound + p.G) - 16 : -1;
-            const float sc_next = sc1;
-            sc1 = sc2;
-            sc2 = sc3;
-            sc3 = scale_of(g_idx + 4);
+            const float sc = fscale * __half2float(__ushort_as_half(sr[0]));
+#pragma unroll
+            for (int j = 0; j < kSR - 1; ++j) sr[j] = sr[j + 1];
+            sr[kSR - 1] = scale_raw(g_idx + kSR);
             const int db = sg % DB;
             const bool okw = ptx::mbar_wait(ptx::smem_addr(&bar_dfull[db]), (sg / DB) & 1, &s_abort, p.wait_ns);
             if (!__all_sync(0xffffffffu, okw)) {  // warp-uniform: tcgen05.ld is .sync.aligned
@@ -540,7 +547,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             ptx::mbar_arrive(ptx::smem_addr(&bar_dempty[db]));
             ++sg;
             k_end = k_next;
-            sc = sc_next;
             ++g_idx;
             bound += p.G;
         }
