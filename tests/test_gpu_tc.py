@@ -64,9 +64,11 @@ def test_tc_group_sizes_and_splits(w, G, split):
     assert_close(run(w, c, kernel=w.KERNEL_TC, split_k=split), ref(c), f"TC G={G} split={split}")
 
 
+@pytest.mark.parametrize("M", [32, 96, 128])
 @pytest.mark.parametrize("split", [2, 5, 7, 16])
-def test_tc_splits(w, split):
-    c = synth.make_case(32, 2048, 1024, 128, sym=True, seed=split)
+def test_tc_splits(w, split, M):
+    # 96 and 128 rows: two epilogue warpgroups, each reducing its half of the rows
+    c = synth.make_case(M, 2048, 1024, 128, sym=True, seed=split)
     assert_close(run(w, c, kernel=w.KERNEL_TC, split_k=split), ref(c), f"TC split={split}")
 
 

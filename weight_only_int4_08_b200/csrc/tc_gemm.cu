@@ -75,8 +75,15 @@ __host__ __device__ constexpr int deq_warps(int mn) { return mn <= 64 ? 8 : 4; }
 // Weight producers: stage i of the weight ring is issued by producer i % P (one: measured on
 // B200 at M = 32, four issuing warps did not raise the weight rate).
 __host__ __device__ constexpr int wproducer_warps(int mn) { return (void)mn, 1; }
-// Warps: dequantisers, weight producers, an activation producer, the MMA issuer, four epilogue warps.
-__host__ __device__ constexpr int tc_threads(int mn) { return (deq_warps(mn) + wproducer_warps(mn) + 6) * 32; }
+// Epilogue warps: one warpgroup, or two above 32 rows that split the accumulator's columns (rows of
+// A) between them. Each epilogue thread loads its share of every group's accumulator from TMEM (16
+// columns per load and wait) and adds it, scaled, to per-row totals in registers; measured on B200
+// (M = 128, dequantisers and MMAs doing no work), one warpgroup spent ~0.7 us per group on it.
+__host__ __device__ constexpr int epi_warps(int mn) { return mn >= 64 && mn % 32 == 0 ? 8 : 4; }
+// Warps: dequantisers, weight producers, an activation producer, the MMA issuer, the epilogue.
+__host__ __device__ constexpr int tc_threads(int mn) {
+    return (deq_warps(mn) + wproducer_warps(mn) + 2 + epi_warps(mn)) * 32;
+}
 
 template <int MN>
 struct TcCfg {
@@ -155,6 +162,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     constexpr int kWProducers = wproducer_warps(MN);
     constexpr int kWProducer = kDeqWarps, kAProducer = kDeqWarps + kWProducers, kMmaWarp = kAProducer + 1,
                   kEpiWarp0 = kMmaWarp + 1;
+    constexpr int kEpiWarps = epi_warps(MN), kEpiThreads = 32 * kEpiWarps;
+    constexpr int EH = MN / (kEpiWarps / 4);   // accumulator columns (rows of A) per epilogue warpgroup
     constexpr int WS = C::kWStages, AS = C::kAStages;
     static_assert(WS % kWProducers == 0, "every weight slot has one producer");
     extern __shared__ __align__(1024) unsigned char s_raw[];
@@ -195,7 +204,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         }
         for (int i = 0; i < DB; ++i) {
             ptx::mbar_init(ptx::smem_addr(&bar_dfull[i]), 1);
-            ptx::mbar_init(ptx::smem_addr(&bar_dempty[i]), 128);
+            ptx::mbar_init(ptx::smem_addr(&bar_dempty[i]), 32 * kEpiWarps);
         }
         ptx::mbar_init(ptx::smem_addr(&bar_drain), 1);
         ptx::mbar_fence_init();
@@ -494,13 +503,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     } else {
         // -------------------------------------------------------------- epilogue
         const int sub = warp & 3;                           // TMEM lanes 32 sub .. 32 sub + 31
-        const int et = threadIdx.x - 32 * kEpiWarp0;        // 0..127 within the epilogue warps
+        const int et = threadIdx.x - 32 * kEpiWarp0;        // index within the epilogue warps
+        const int m0 = (et / 128) * EH;                     // my warpgroup's first accumulator column
         const int ncol = 32 * sub + 4 * (lane & 7) + (lane >> 3);
         const int64_t n = (int64_t)tile * kBlockN + ncol;
         const float fscale = (lane >> 3) & 1 ? 0.0625f : 1.0f;
-        float tot[MN];
+        float tot[EH];
 #pragma unroll
-        for (int m = 0; m < MN; ++m) tot[m] = 0.f;
+        for (int m = 0; m < EH; ++m) tot[m] = 0.f;
         int sg = 0;
         bool ok = true;
         // Segment ends in order (group boundaries, tracked incrementally).
@@ -534,9 +544,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 break;
             }
             ptx::tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(C::kDCol + db * MN);
+            const uint32_t taddr = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(C::kDCol + db * MN + m0);
 #pragma unroll
-            for (int c0 = 0; c0 < MN; c0 += 16) {
+            for (int c0 = 0; c0 < EH; c0 += 16) {
                 uint32_t v[16];
                 ptx::tmem_ld_32x32b_x16(taddr + c0, v);
                 ptx::tmem_wait_ld();
@@ -550,29 +560,29 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             ++g_idx;
             bound += p.G;
         }
-        // One decision for all 128 epilogue threads (a timeout seen by any of them,
+        // One decision for all epilogue threads (a timeout seen by any of them,
         // or by another role, skips the output), so the named barriers below match.
-        const bool bad = ptx::named_bar_or(1, 128, !ok || s_abort);
+        const bool bad = ptx::named_bar_or(1, kEpiThreads, !ok || s_abort);
         asm volatile("griddepcontrol.wait;" ::: "memory");   // before the first write
         if (!bad) {
             if (p.split == 1) {
 #pragma unroll
-                for (int m = 0; m < MN; ++m)
-                    if (m < p.mblk) p.out.put((int64_t)m * p.N + n, tot[m]);
+                for (int m = 0; m < EH; ++m)
+                    if (m0 + m < p.mblk) p.out.put((int64_t)(m0 + m) * p.N + n, tot[m]);
             } else {
 #pragma unroll
-                for (int m = 0; m < MN; ++m)
-                    if (m < p.mblk) p.partials[((int64_t)blockIdx.y * p.mblk + m) * p.N + n] = tot[m];
+                for (int m = 0; m < EH; ++m)
+                    if (m0 + m < p.mblk) p.partials[((int64_t)blockIdx.y * p.mblk + m0 + m) * p.N + n] = tot[m];
                 __threadfence();
-                ptx::named_bar_sync(1, 128);
+                ptx::named_bar_sync(1, kEpiThreads);
                 if (et == 0) {
                     const uint32_t ticket = atomicAdd(p.counters + tile, 1u);
                     s_last = (ticket == (uint32_t)p.split - 1);
                 }
-                ptx::named_bar_sync(1, 128);
+                ptx::named_bar_sync(1, kEpiThreads);
                 if (s_last) {
                     __threadfence();
-                    for (int m = 0; m < p.mblk; ++m) {
+                    for (int m = m0; m < min(m0 + EH, p.mblk); ++m) {
                         float a = 0.f;
                         for (int y = 0; y < p.split; ++y) a += __ldcg(p.partials + ((int64_t)y * p.mblk + m) * p.N + n);
                         p.out.put((int64_t)m * p.N + n, a);
