@@ -67,11 +67,13 @@ constexpr int kBoxes = kStageK / kBoxK;         // activation boxes per stage
 constexpr int kMmaPerStage = kStageK / 16;      // K = 16 per tcgen05.mma.kind::f16
 constexpr int kAColsPerStage = kStageK / 2;     // TMEM columns of one A slot (two fp16 per column)
 constexpr int kTmemStages = 4;                  // A slots in TMEM
-// Dequantiser warps: groups of four (one per TMEM lane quarter) that take turns on the stages,
-// two groups while the MMAs are short (MN <= 64), one above, where the per-column totals of
-// the epilogue need the registers that more threads would take. A group's stage ends with a
-// wait for its TMEM stores; a second group keeps another stage in flight meanwhile.
-__host__ __device__ constexpr int deq_warps(int mn) { return mn <= 64 ? 8 : 4; }
+// Dequantiser warps: groups of four (one per TMEM lane quarter) that take turns on the stages. A
+// group's stage ends with a wait for its TMEM stores; a second group keeps another stage in flight
+// meanwhile. Two groups, except at MN = 112, where one epilogue warpgroup holds 112 totals per
+// thread and more threads would leave too few registers. Measured on B200 (K=4096, N=14336,
+// PDL): M = 128 33.4 -> 27.9 us with two groups (and the two epilogue warpgroups below).
+__host__ __device__ constexpr int epi_warps(int mn);
+__host__ __device__ constexpr int deq_warps(int mn) { return mn <= 80 || epi_warps(mn) == 8 ? 8 : 4; }
 // Weight producers: stage i of the weight ring is issued by producer i % P (one: measured on
 // B200 at M = 32, four issuing warps did not raise the weight rate).
 __host__ __device__ constexpr int wproducer_warps(int mn) { return (void)mn, 1; }
