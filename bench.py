@@ -184,16 +184,16 @@ class Problem:
         # The library's automatic choice: tensor-core GEMM (one launch per 128 rows) above 32 rows,
         # and for 17..32 rows when N has at least 96 tiles of 128 columns; otherwise the GEMV (one
         # launch per 16 rows).
-        return (self.M + 127) // 128 if uses_tc(self.M, self.N) else (self.M + 15) // 16
+        return (self.M + 127) // 128 if uses_tc(self.M, self.N, self.K) else (self.M + 15) // 16
 
 
 def copies_for(bytes_per_copy):
     return max(2, int(np.ceil(2 * L2_BYTES / bytes_per_copy)) + 1)
 
 
-def uses_tc(M, N):
+def uses_tc(M, N, K=4096):
     """The library's automatic kernel choice for an aligned problem (see w4a16_api.cu)."""
-    return M > 32 or (M > 16 and N // 128 >= 96)
+    return M > 32 or (M > 16 and (N // 128 >= 96 or K >= 8192))
 
 
 def capture(torch, fn, n):

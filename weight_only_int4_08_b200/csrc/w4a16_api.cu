@@ -83,17 +83,18 @@ struct Choice {
 
 // Kernel table. M <= 16: the mma.sync GEMV (one launch; the CUDA-core GEMV when its
 // alignment rules fail). 17..32 rows: the GEMV needs two launches, each reading all the
-// weights, while the tensor-core GEMM reads them once, one CTA per 128 columns; the GEMM is
-// taken when N has at least 96 such column tiles. Above 32 rows: the GEMM. The GEMM only
-// when the shape and pointers allow it (N % 128, K % 128, 16-byte aligned A and weights),
-// the GEMV's row blocks otherwise. Null pointers (workspace query) count as aligned.
-// Measured on B200 at M=32, G=128, CUDA graphs, weights larger than L2 (GEMV / GEMM):
-// K=4096 N=14336 37.6 / 20.6 us; N=28672 72.7 / 41.2 us; N=6144 31.8 / 33.0 us;
-// N=4096 25.8 / 25.8 us; K=14336 N=4096 41.5 / 36.2 us. At K=4096 N=14336 the GEMM is
-// ahead from 17 rows (31.2 / 19.8 us).
-constexpr int64_t kGemvOneLaunchM = 16, kGemvMaxM = 32, kTcMinTiles = 96;
-bool auto_prefers_tc(int64_t M, int64_t N) {
-    return M > kGemvMaxM || (M > kGemvOneLaunchM && N / 128 >= kTcMinTiles);
+// weights, while the tensor-core GEMM reads them once, one CTA per 128 columns (times a K
+// split); the GEMM is taken when N has at least 96 such column tiles, or when K is at least
+// 8192 (a long K splits into enough CTAs). Above 32 rows: the GEMM. The GEMM only when the
+// shape and pointers allow it (N % 128, K % 128, 16-byte aligned A and weights), the GEMV's
+// row blocks otherwise. Null pointers (workspace query) count as aligned.
+// Measured on B200 at M=32, G=128, CUDA graphs with programmatic dependent launch, weights
+// larger than L2 (GEMV / GEMM): K=4096 N=14336 32.3 / 19.2 us; N=28672 71.8 / 38.3 us;
+// N=6144 29.3 / 32.2 us; N=4096 24.2 / 25.2 us; K=14336 N=4096 39.9 / 34.4 us. At 24 rows
+// the narrow K=4096 layers are within 10 % either way (N=6144 27.7 / 26.3 us).
+constexpr int64_t kGemvOneLaunchM = 16, kGemvMaxM = 32, kTcMinTiles = 96, kTcMinK = 8192;
+bool auto_prefers_tc(int64_t M, int64_t N, int64_t K) {
+    return M > kGemvMaxM || (M > kGemvOneLaunchM && (N / 128 >= kTcMinTiles || K >= kTcMinK));
 }
 Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms,
               const void* a, const void* b, const void* s, const void* z) {
@@ -102,7 +103,7 @@ Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_optio
     const bool tc_ok = tc_supported(M, N, K, G, a ? a : (const void*)16, b ? b : (const void*)16);
     if (req == W4A16_KERNEL_TC) c.kernel = W4A16_KERNEL_TC;
     else if (req == W4A16_KERNEL_GEMV || req == W4A16_KERNEL_GEMV_FMA) c.kernel = W4A16_KERNEL_GEMV;
-    else c.kernel = (auto_prefers_tc(M, N) && tc_ok) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
+    else c.kernel = (auto_prefers_tc(M, N, K) && tc_ok) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
     const int split = opts ? opts->split_k : 0;
     if (c.kernel == W4A16_KERNEL_TC) {
         if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, split);
@@ -127,7 +128,7 @@ size_t ws_bound(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_opt
         if (req != W4A16_KERNEL_GEMV_FMA && N % 32 == 0) ws = std::max(ws, plan_gemv_mma(M, N, K, G, split, sms).ws_bytes);
     }
     const bool tc_shape = tc_supported(M, N, K, G, (const void*)16, (const void*)16);
-    if (tc_shape && (req == W4A16_KERNEL_TC || (req == W4A16_KERNEL_AUTO && auto_prefers_tc(M, N))))
+    if (tc_shape && (req == W4A16_KERNEL_TC || (req == W4A16_KERNEL_AUTO && auto_prefers_tc(M, N, K))))
         ws = std::max(ws, plan_tc(M, N, K, G, sms, opts ? opts->split_k : 0).ws_bytes);
     return ws;
 }
@@ -258,7 +259,7 @@ w4a16_status w4a16_gemm_kernel_choice(int64_t M, int64_t N, int64_t K, int32_t g
     const void* pb = b_packed ? b_packed : (const void*)16;
     const void* ps = scales ? scales : (const void*)16;
     // the same decisions as choose() and the launch path, without the device queries
-    if (auto_prefers_tc(M, N) && tc_supported(M, N, K, group_size, pa, pb))
+    if (auto_prefers_tc(M, N, K) && tc_supported(M, N, K, group_size, pa, pb))
         *kernel = W4A16_KERNEL_TC;
     else
         *kernel = gemv_mma_supported(N, K, pa, pb, ps, nullptr) ? W4A16_KERNEL_GEMV : W4A16_KERNEL_GEMV_FMA;
