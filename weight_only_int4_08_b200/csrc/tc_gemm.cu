@@ -77,11 +77,12 @@ __host__ __device__ constexpr int deq_warps(int mn) { return mn <= 80 || epi_war
 // Weight producers: stage i of the weight ring is issued by producer i % P (one: measured on
 // B200 at M = 32, four issuing warps did not raise the weight rate).
 __host__ __device__ constexpr int wproducer_warps(int mn) { return (void)mn, 1; }
-// Epilogue warps: one warpgroup, or two above 32 rows that split the accumulator's columns (rows of
-// A) between them. Each epilogue thread loads its share of every group's accumulator from TMEM (16
-// columns per load and wait) and adds it, scaled, to per-row totals in registers; measured on B200
-// (M = 128, dequantisers and MMAs doing no work), one warpgroup spent ~0.7 us per group on it.
-__host__ __device__ constexpr int epi_warps(int mn) { return mn >= 64 && mn % 32 == 0 ? 8 : 4; }
+// Epilogue warps: one warpgroup, or two (MN = 32, 64, 96, 128) that split the accumulator's
+// columns (rows of A) between them. Each epilogue thread loads its share of every group's
+// accumulator from TMEM (16 columns per load and wait) and adds it, scaled, to per-row totals in
+// registers; measured on B200 (M = 128, dequantisers and MMAs doing no work), one warpgroup spent
+// ~0.7 us per group on it. At M = 32 two warpgroups save ~0.6 us per call.
+__host__ __device__ constexpr int epi_warps(int mn) { return mn >= 32 && mn % 32 == 0 ? 8 : 4; }
 // Warps: dequantisers, weight producers, an activation producer, the MMA issuer, the epilogue.
 __host__ __device__ constexpr int tc_threads(int mn) {
     return (deq_warps(mn) + wproducer_warps(mn) + 2 + epi_warps(mn)) * 32;
