@@ -102,9 +102,11 @@ __host__ __device__ constexpr int tot_per_tile(int mt) { return mt > 1 ? 8 : 4; 
 __host__ __device__ constexpr int tot_per_chunk(int mt) { return tot_per_tile(mt) * n_tiles(mt); }
 // Dynamic shared memory: weight ring, activation ring, fp32 totals, group buffers, and the
 // warp-reduced sums of the (at most two) fragments shared with other CTAs.
-__host__ __device__ constexpr size_t sk_smem_bytes(int warps, int mt) {
+// recv: the launch's layout splits tiles between CTAs, whose owners receive the other parts.
+__host__ __device__ constexpr size_t sk_smem_bytes(int warps, int mt, bool recv = false) {
     return (size_t)warps * kRing * (wstage_bytes(mt) + a_slot_bytes(mt)) +
-           (size_t)warps * 4 * tot_per_chunk(mt) * 32 * 4 + (size_t)warps * 2 * kGrpBytes + 2 * (size_t)mt * kTileN * 4;
+           (size_t)warps * 4 * tot_per_chunk(mt) * 32 * 4 + (size_t)warps * 2 * kGrpBytes + 2 * (size_t)mt * kTileN * 4 +
+           (recv ? (size_t)(kMaxCluster - 1) * mt * kTileN * 4 : 0);
 }
 
 struct SkArgs {
@@ -176,6 +178,15 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -221,6 +232,8 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     float* tots = reinterpret_cast<float*>(aring + kWarps * kRing * kASlot);  // [warp][c * NI + i][lane]
     unsigned char* grps = reinterpret_cast<unsigned char*>(tots + kWarps * 4 * NI * 32);  // [warp][2][kGrpBytes]
     float* keep = reinterpret_cast<float*>(grps + kWarps * 2 * kGrpBytes);                // [2][MT][128]
+    float* recv = keep + 2 * MT * kTileN;   // [kMaxCluster - 1][MT][128]: parts of a shared tile I own
+                                            // (allocated when the layout shares tiles)
     __shared__ __align__(8) uint64_t s_full[kWarps][kRing];
     __shared__ __align__(16) uint4 s_zero;   // the B rows past MT read these zeros
     __shared__ volatile int s_abort;
@@ -258,6 +271,15 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         ptx::mbar_fence_init();
     }
     __syncthreads();
+    // Shared tiles: the CTAs that share a tile with its first (owning) CTA store their parts into
+    // the owner's shared memory before the cluster barrier at the end, and the owner adds them up
+    // after it; nobody reads another CTA's shared memory, so nobody waits for another to finish
+    // reading. Remote stores need the owner to have started: every CTA arrives here and waits (after
+    // its first loads, by when all have arrived) before its first remote store. Every CTA of a
+    // cluster computes the same cluster_shares, so all of them or none take the cluster barriers.
+    const bool cluster_shares =
+        (tile_hi - tile_lo == p.tiles_per_cluster ? p.shares_mask & 1 : p.shares_mask & 2) != 0;
+    if (cluster_shares) cluster_arrive_relaxed();
 
     // Per-warp shared-memory addresses of ring slot 0 (slot j adds j times the slot size).
     const uint32_t bar0 = ptx::smem_addr(&s_full[warp][0]);
@@ -303,6 +325,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         for (int j = 0; j < kRing; ++j) first_kb[j] = arm_w();
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (cluster_shares) cluster_wait();   // every CTA of the cluster has started
     if (lane == 0 && !p.stall_loads) {
 #pragma unroll
         for (int j = 0; j < kRing; ++j)
@@ -521,8 +544,13 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         __syncthreads();
         // s_abort is read by every thread between two barriers with no wait in between: uniform.
         if (s_abort == 0) {
-            const bool shared_tile = rank_of(tile * nblk - ubase, U, S) != rank_of((tile + 1) * nblk - 1 - ubase, U, S);
+            const int first = rank_of(tile * nblk - ubase, U, S);
+            const bool shared_tile = first != rank_of((tile + 1) * nblk - 1 - ubase, U, S);
             float* kp = keep + (f == 0 ? 0 : MT * kTileN);
+            // a part for the owner: slot rank - first - 1 of its receive buffer
+            const uint32_t rp = shared_tile && first != rank
+                                    ? map_rank(ptx::smem_addr(recv + (rank - first - 1) * MT * kTileN), (uint32_t)first)
+                                    : 0u;
             for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
                 const int m = item / kTileN, nl = item % kTileN;
                 const int64_t n = (int64_t)tile * kTileN + nl;
@@ -534,23 +562,25 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
                 float v = 0.f;
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) v += tots[w * 4 * NI * 32 + src];
-                if (shared_tile) kp[item] = v;
-                else if (n < p.N) p.out.put((int64_t)m * p.N + n, v);
+                if (!shared_tile) {
+                    if (n < p.N) p.out.put((int64_t)m * p.N + n, v);
+                } else if (first == rank) {
+                    kp[item] = v;
+                } else {
+                    st_cluster(rp + 4 * item, v);
+                }
             }
         }
         __syncthreads();  // the totals are free again
     }
 
-    // ---- tiles shared within the cluster: the first CTA touching a tile sums every part, in rank
-    // order, from the CTAs' shared memory (distributed shared memory), then writes the tile ----
+    // ---- tiles shared within the cluster: the first CTA touching a tile adds its own part and the
+    // parts the others stored into its receive buffer, in rank order, then writes the tile ----
     // Only a cluster whose rank boundaries cut through a tile has shared tiles; the others (every CTA
-    // runs whole tiles) neither read each other's shared memory nor wait for each other. Every CTA
-    // of a cluster computes the same answer, so all of them or none take the cluster barriers.
-    // Measured on B200 (decode GEMV, clusters of 3 CTAs over 3 tiles): the two barriers cost a CTA
-    // ~1.6 us at the end of the launch.
-    const bool cluster_shares =
-        (tile_hi - tile_lo == p.tiles_per_cluster ? p.shares_mask & 1 : p.shares_mask & 2) != 0;
-    if (cluster_shares) cluster_sync();
+    // runs whole tiles) take no cluster barrier. Measured on B200: the two barriers of the earlier
+    // exchange (read the parts remotely, then wait for every reader) cost a CTA ~1.6 us at the end
+    // of a decode launch; this one has a single barrier, after which only the owners work.
+    if (cluster_shares) cluster_sync();   // every part has been stored (release / acquire)
     if (cluster_shares && s_abort == 0) {
 #pragma unroll
         for (int d = 0; d < 2; ++d) {
@@ -558,22 +588,18 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             const int tile = t0 + (d == 0 ? 0 : nfrag - 1);
             const int first = rank_of(tile * nblk - ubase, U, S), last = rank_of((tile + 1) * nblk - 1 - ubase, U, S);
             if (first == last || first != rank) continue;
-            uint32_t src[kMaxCluster];   // keep slot of this tile in each contributing CTA (first tile of its run: 0)
-            for (int rr = first; rr <= last; ++rr) {
-                const int first_tile_rr = (ubase + (int)((int64_t)U * rr / S)) / nblk;
-                src[rr - first] = map_rank(ptx::smem_addr(keep + (tile == first_tile_rr ? 0 : MT * kTileN)), (uint32_t)rr);
-            }
+            const float* own = keep + (d == 0 ? 0 : MT * kTileN);
             for (int item = threadIdx.x; item < MT * kTileN; item += kThreads) {
                 const int m = item / kTileN, nl = item % kTileN;
                 const int64_t n = (int64_t)tile * kTileN + nl;
                 if (n >= p.N) continue;
                 float v = 0.f;
-                for (int rr = first; rr <= last; ++rr) v += ld_cluster(src[rr - first] + 4 * item);
+                v += own[item];
+                for (int rr = first + 1; rr <= last; ++rr) v += recv[(rr - first - 1) * MT * kTileN + item];
                 p.out.put((int64_t)m * p.N + n, v);
             }
         }
     }
-    if (cluster_shares) cluster_sync();   // no CTA leaves while another still reads its shared memory
 
     // A wait gave up: let the copies already issued land before the CTA's shared memory goes away.
     cp_async_wait_all();
@@ -810,7 +836,7 @@ cudaError_t launch_gemv_mma(const __half* a, const uint32_t* b, const __half* s,
         }
         args.stall_loads = wp.stall_loads;
         args.wait_ns = wp.limit_ns;
-        const size_t smem = sk_smem_bytes(l.warps, mt);
+        const size_t smem = sk_smem_bytes(l.warps, mt, args.shares_mask != 0);
         SkFn k = select_sk(l.warps, mt, G % rows == 0);
         cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
