@@ -569,9 +569,36 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         asm volatile("griddepcontrol.wait;" ::: "memory");   // before the first write
         if (!bad) {
             if (p.split == 1) {
+                // The tile goes out through shared memory: every stage has been consumed (the last
+                // group's accumulator is complete, so every MMA, and before them every dequantiser
+                // read and every load, has finished), so the weight ring is idle. Each thread puts its
+                // column there row-major, then whole rows leave as 16-byte stores. Measured on B200
+                // (M = 128), one 2-byte store per row and thread took ~3.9 us at the end of the launch.
+                const bool f32 = p.out.f != nullptr;
+                const int esz = f32 ? 4 : 2;
+                unsigned char* stg = s_w;
 #pragma unroll
-                for (int m = 0; m < EH; ++m)
-                    if (m0 + m < p.mblk) p.out.put((int64_t)(m0 + m) * p.N + n, tot[m]);
+                for (int m = 0; m < EH; ++m) {
+                    if (f32) reinterpret_cast<float*>(stg)[(m0 + m) * kBlockN + ncol] = tot[m];
+                    else reinterpret_cast<__half*>(stg)[(m0 + m) * kBlockN + ncol] = __float2half_rn(tot[m]);
+                }
+                ptx::named_bar_sync(1, kEpiThreads);
+                unsigned char* obase = f32 ? reinterpret_cast<unsigned char*>(p.out.f) : reinterpret_cast<unsigned char*>(p.out.h);
+                const int64_t row_stride = p.N * esz, col0 = (int64_t)tile * kBlockN * esz;
+                if (((reinterpret_cast<uintptr_t>(obase) | (uintptr_t)row_stride) & 15) == 0) {
+                    const int cpr = kBlockN * esz / 16;   // 16-byte chunks per row of the tile
+                    for (int c = et; c < p.mblk * cpr; c += kEpiThreads) {
+                        const int r = c / cpr, q = c % cpr;
+                        const uint4 v = *reinterpret_cast<const uint4*>(stg + r * kBlockN * esz + q * 16);
+                        *reinterpret_cast<uint4*>(obase + r * row_stride + col0 + q * 16) = v;
+                    }
+                } else {
+                    for (int c = et; c < p.mblk * kBlockN; c += kEpiThreads) {
+                        const int r = c / kBlockN, q = c % kBlockN;
+                        if (f32) p.out.f[(int64_t)r * p.N + (int64_t)tile * kBlockN + q] = reinterpret_cast<const float*>(stg)[c];
+                        else p.out.h[(int64_t)r * p.N + (int64_t)tile * kBlockN + q] = reinterpret_cast<const __half*>(stg)[c];
+                    }
+                }
             } else {
 #pragma unroll
                 for (int m = 0; m < EH; ++m)
