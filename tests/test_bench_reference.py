@@ -30,3 +30,13 @@ def test_reference_arm_prints_the_contract_line():
 
 def test_reference_arm_other_ranks_exit_quietly():
     assert _run({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_cpu_baseline_takes_a_checkpoint_layout_case():
+    """The batch workload draws its weights in the checkpoint layout; the baseline repacks them."""
+    import bench
+    import synth
+    c = synth.make_case(4, 256, 64, 64, sym=False, seed=5, ckpt_layout=True)
+    assert c.get("b") is None
+    r = bench.cpu_baseline(c, seconds=0.01)
+    assert r["kind"] == "oracle" and r["value"] > 0 and "M=4 K=256 N=64" in r["sample"]
