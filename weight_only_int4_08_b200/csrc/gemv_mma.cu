@@ -251,7 +251,11 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     const int tile_lo = (int)(blockIdx.x / S) * p.tiles_per_cluster;
     const int tile_hi = min(tile_lo + p.tiles_per_cluster, p.tiles);
     const int ubase = tile_lo * nblk, U = (tile_hi - tile_lo) * nblk;
-    const int u0 = ubase + (int)((int64_t)U * rank / S), u1 = ubase + (int)((int64_t)U * (rank + 1) / S);
+    // (32-bit arithmetic unless a cluster holds 2^29 units or more)
+    auto split_at = [&](int r) -> int {
+        return U < (1 << 29) ? (int)((uint32_t)U * (uint32_t)r / (uint32_t)S) : (int)((int64_t)U * r / S);
+    };
+    const int u0 = ubase + split_at(rank), u1 = ubase + split_at(rank + 1);
     const int t0 = u0 / nblk;
     const int nfrag = u1 > u0 ? (u1 - 1) / nblk - t0 + 1 : 0;
 
@@ -263,14 +267,18 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         hi = a + (b - a) * (warp + 1) / kWarps;
     };
 
+    // Each warp's ring is waited on by that warp alone: its lane 0 initialises the ring's barriers and
+    // issues the first loads before the block-wide barrier, which only the abort flag and the zero row
+    // need (neither is read before it).
     if (threadIdx.x == 0) {
         s_abort = 0;
         s_zero = make_uint4(0u, 0u, 0u, 0u);
-        for (int w = 0; w < kWarps; ++w)
-            for (int j = 0; j < kRing; ++j) ptx::mbar_init(ptx::smem_addr(&s_full[w][j]), 1);
+    }
+    if (lane == 0) {
+        for (int j = 0; j < kRing; ++j) ptx::mbar_init(ptx::smem_addr(&s_full[warp][j]), 1);
         ptx::mbar_fence_init();
     }
-    __syncthreads();
+    __syncwarp();
     // Shared tiles: the CTAs that share a tile with its first (owning) CTA store their parts into
     // the owner's shared memory before the cluster barrier at the end, and the owner adds them up
     // after it; nobody reads another CTA's shared memory, so nobody waits for another to finish
@@ -279,7 +287,6 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
     // cluster computes the same cluster_shares, so all of them or none take the cluster barriers.
     const bool cluster_shares =
         (tile_hi - tile_lo == p.tiles_per_cluster ? p.shares_mask & 1 : p.shares_mask & 2) != 0;
-    if (cluster_shares) cluster_arrive_relaxed();
 
     // Per-warp shared-memory addresses of ring slot 0 (slot j adds j times the slot size).
     const uint32_t bar0 = ptx::smem_addr(&s_full[warp][0]);
@@ -324,6 +331,8 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
         for (int j = 0; j < kRing; ++j) first_kb[j] = arm_w();
     }
+    __syncthreads();   // the abort flag and the zero row are set
+    if (cluster_shares) cluster_arrive_relaxed();
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (cluster_shares) cluster_wait();   // every CTA of the cluster has started
     if (lane == 0 && !p.stall_loads) {
