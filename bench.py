@@ -193,7 +193,7 @@ def copies_for(bytes_per_copy):
 
 def uses_tc(M, N, K=4096):
     """The library's automatic kernel choice for an aligned problem (see w4a16_api.cu)."""
-    return M > 32 or (M > 16 and (N // 128 >= 96 or K >= 8192))
+    return M > 24 or (M > 16 and N // 128 >= 96)
 
 
 def capture(torch, fn, n):

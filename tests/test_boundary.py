@@ -170,13 +170,14 @@ KERNELS = {"GEMV": 1, "TC": 2, "GEMV_FMA": 3}
     (16, 14336, 4096, 128, {}, "GEMV"),          # one GEMV launch
     (17, 14336, 4096, 128, {}, "TC"),            # 112 column tiles >= 96
     (32, 14336, 4096, 128, {}, "TC"),
-    (32, 6144, 4096, 128, {}, "GEMV"),           # 48 column tiles
-    (32, 12288, 4096, 128, {}, "TC"),            # exactly 96
-    (32, 12160, 4096, 128, {}, "GEMV"),          # 95
-    (32, 4096, 14336, 128, {}, "TC"),            # K >= 8192: a long K splits into enough CTAs
-    (17, 4096, 8192, 128, {}, "TC"),
-    (32, 4096, 8064, 128, {}, "GEMV"),           # K < 8192 on a narrow layer
-    (33, 4096, 4096, 128, {}, "TC"),             # above 32 rows: the GEMM whenever it can
+    (24, 6144, 4096, 128, {}, "GEMV"),           # 48 column tiles
+    (25, 6144, 4096, 128, {}, "TC"),             # above 24 rows: the GEMM whenever it can
+    (24, 12288, 4096, 128, {}, "TC"),            # exactly 96
+    (24, 12160, 4096, 128, {}, "GEMV"),          # 95
+    (24, 4096, 14336, 128, {}, "GEMV"),          # a long K alone does not take the GEMM
+    (28, 4096, 14336, 128, {}, "TC"),
+    (32, 4096, 8064, 128, {}, "TC"),
+    (33, 4096, 4096, 128, {}, "TC"),
     (64, 4096, 4160, 64, {}, "GEMV"),            # K % 128 != 0
     (64, 4128, 4096, 128, {}, "GEMV"),           # N % 128 != 0, N % 32 == 0
     (64, 4104, 4096, 128, {}, "GEMV_FMA"),       # N % 32 != 0
@@ -193,7 +194,7 @@ def test_kernel_choice_table(M, N, K, G, ptrs, expect):
 
 def test_kernel_choice_agrees_with_the_bench():
     import bench
-    for M in (1, 8, 16, 17, 24, 32, 33, 64, 128):
+    for M in (1, 8, 16, 17, 24, 25, 32, 33, 64, 128):
         for N in (4096, 6144, 12160, 12288, 14336, 28672):
             for K in (4096, 8064, 8192, 14336):
                 k = w.w4a16_gemm_kernel_choice(M, N, K, 128)

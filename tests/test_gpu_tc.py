@@ -38,7 +38,7 @@ def test_config4_m32_tensor_cores(w):
     assert_close(run(w, c, b=b_dev, kernel=w.KERNEL_TC), ref(c), "config4 TC")
 
 
-@pytest.mark.parametrize("M", [1, 5, 9, 17, 31, 33, 48, 64, 100, 128, 129, 200])
+@pytest.mark.parametrize("M", [1, 5, 9, 17, 31, 33, 40, 48, 64, 72, 100, 112, 128, 129, 200])
 def test_tc_row_blocks(w, M):
     c = synth.make_case(M, 512, 384, 128, sym=(M % 2 == 0), seed=100 + M)
     assert_close(run(w, c, kernel=w.KERNEL_TC), ref(c), f"TC M={M}")
@@ -64,10 +64,11 @@ def test_tc_group_sizes_and_splits(w, G, split):
     assert_close(run(w, c, kernel=w.KERNEL_TC, split_k=split), ref(c), f"TC G={G} split={split}")
 
 
-@pytest.mark.parametrize("M", [32, 96, 128])
+@pytest.mark.parametrize("M", [32, 40, 72, 96, 104, 128])
 @pytest.mark.parametrize("split", [2, 5, 7, 16])
 def test_tc_splits(w, split, M):
-    # 96 and 128 rows: two epilogue warpgroups, each reducing its half of the rows
+    # From 32 rows up two epilogue warpgroups each reduce their half of the rows; at 40, 72 and
+    # 104 rows (tile widths 48, 80, 112) the halves are 24, 40 and 56 columns wide.
     c = synth.make_case(M, 2048, 1024, 128, sym=True, seed=split)
     assert_close(run(w, c, kernel=w.KERNEL_TC, split_k=split), ref(c), f"TC split={split}")
 

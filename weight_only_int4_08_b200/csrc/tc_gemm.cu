@@ -12,33 +12,34 @@
 // sum D_g is exact up to fp32 summation; the fp16 scale is applied in fp32 when
 // D_g is read back (tot += s[g, n] * D_g), never rounded into the weights.
 //
-// Roles (one CTA = one 128-column tile x one K slab; 14 warps, 10 above MN = 64;
-// the warp numbers below are those of the 14-warp form):
-//   warp 8      producer: per stage of 128 k-rows, one 2-D TMA load of the
-//               tile's packed words [128 rows x 64 B] (64-byte swizzle) and two of
-//               the activation tile [MN x 64] (128-byte swizzle, the canonical
-//               K-major layout of operand B), into an 8-stage ring (4 above
-//               MN = 64);
-//   warps 0-7   dequantisers (0-3 above MN = 64): warp p owns TMEM lanes
-//               32(p%4)..+31 and tile columns 32(p%4)..+31 (one 16-byte chunk of
-//               each weight row); warps 0-3 take the even stages and 4-7 the odd
-//               ones; ldmatrix.trans hands every thread two k-rows of 4 columns
-//               per register, which become exact fp16 (q - z) pairs (0x6400 magic
-//               + fp16 subtract) written to TMEM with tcgen05.st.16x128b.x4;
-//   warp 9      TMEM allocator and MMA issuer: tcgen05.mma.kind::f16 with A
+// Roles (one CTA = one 128-column tile x one K slab; 19 warps, 15 at MN = 16):
+//   warps 0-7   dequantisers: warp p owns TMEM lanes 32(p%4)..+31 and tile
+//               columns 32(p%4)..+31 (one 16-byte chunk of each weight row);
+//               warps 0-3 take the even stages and 4-7 the odd ones;
+//               ldmatrix.trans hands every thread two k-rows of 4 columns per
+//               register, which become exact fp16 (q - z) pairs (0x6400 magic +
+//               fp16 subtract) written to TMEM with tcgen05.st.16x128b.x4;
+//   warp 8      weight producer: per stage of 128 k-rows, one 2-D TMA load of
+//               the tile's packed words [128 rows x 64 B] (64-byte swizzle) into
+//               a ring of up to 16 stages;
+//   warp 9      activation producer: per stage, two TMA loads of the activation
+//               tile [MN x 64] (128-byte swizzle, the canonical K-major layout of
+//               operand B), into an 8-stage ring (4 above MN = 48);
+//   warp 10     TMEM allocator and MMA issuer: tcgen05.mma.kind::f16 with A
 //               from TMEM and B from shared memory, 8 per stage (K = 16 each);
-//               a fresh accumulator per group segment, double-buffered, and a
-//               tcgen05.commit to an mbarrier at each segment end. When G is a
-//               multiple of 128 (segments are whole stages) the stage loop is
-//               unrolled over the ring so that every operand address is a
-//               constant offset: measured on B200, the issue loop's own
-//               instructions and barrier waits, not the tensor core, set the
+//               a fresh accumulator per group segment, in a ring of TMEM
+//               buffers, and a tcgen05.commit to an mbarrier at each segment
+//               end. When G is a multiple of 128 (segments are whole stages) the
+//               stage loop is unrolled over the ring so that every operand
+//               address is a constant offset: measured on B200, the issue loop's
+//               own instructions and barrier waits, not the tensor core, set the
 //               MMA rate at these small N (about 220 cycles per MMA with per-MMA
 //               bookkeeping, 62 with this form and one wait per stage, 36 for
 //               the MMAs alone at N = 32);
-//   warps 10-13 epilogue: tcgen05.ld of each finished group segment, scaled by
-//               s[g, n] in fp32 into register totals; then the fp16 output, or
-//               the fp32 split-K partial and the last-CTA ordered reduction.
+//   warps 11-18 epilogue (11-14 at MN = 16): tcgen05.ld of each finished group
+//               segment, scaled by s[g, n] in fp32 into register totals; then the
+//               fp16 (or fp32) output, or the fp32 split-K partial and the
+//               last-CTA ordered reduction.
 // Every mbarrier wait is bounded; a wait that runs out sets the workspace
 // status word to W4A16_ERR_TIMEOUT, and all roles drain and leave, freeing TMEM.
 //
@@ -69,20 +70,19 @@ constexpr int kAColsPerStage = kStageK / 2;     // TMEM columns of one A slot (t
 constexpr int kTmemStages = 4;                  // A slots in TMEM
 // Dequantiser warps: groups of four (one per TMEM lane quarter) that take turns on the stages. A
 // group's stage ends with a wait for its TMEM stores; a second group keeps another stage in flight
-// meanwhile. Two groups, except at MN = 112, where one epilogue warpgroup holds 112 totals per
-// thread and more threads would leave too few registers. Measured on B200 (K=4096, N=14336,
-// PDL): M = 128 33.4 -> 27.9 us with two groups (and the two epilogue warpgroups below).
-__host__ __device__ constexpr int epi_warps(int mn);
-__host__ __device__ constexpr int deq_warps(int mn) { return mn <= 80 || epi_warps(mn) == 8 ? 8 : 4; }
+// meanwhile. Measured on B200 (K=4096, N=14336, PDL): M = 128 33.4 -> 27.9 us with two groups
+// (and the two epilogue warpgroups below).
+__host__ __device__ constexpr int deq_warps(int mn) { return (void)mn, 8; }
 // Weight producers: stage i of the weight ring is issued by producer i % P (one: measured on
 // B200 at M = 32, four issuing warps did not raise the weight rate).
 __host__ __device__ constexpr int wproducer_warps(int mn) { return (void)mn, 1; }
-// Epilogue warps: one warpgroup, or two (MN = 32, 64, 96, 128) that split the accumulator's
-// columns (rows of A) between them. Each epilogue thread loads its share of every group's
-// accumulator from TMEM (16 columns per load and wait) and adds it, scaled, to per-row totals in
-// registers; measured on B200 (M = 128, dequantisers and MMAs doing no work), one warpgroup spent
-// ~0.7 us per group on it. At M = 32 two warpgroups save ~0.6 us per call.
-__host__ __device__ constexpr int epi_warps(int mn) { return mn >= 32 && mn % 32 == 0 ? 8 : 4; }
+// Epilogue warps: one warpgroup at MN = 16, else two that split the accumulator's columns (rows
+// of A) into halves of MN / 2. Each epilogue thread loads its share of every group's accumulator
+// from TMEM and adds it, scaled, to per-row totals in registers; measured on B200 (M = 128,
+// dequantisers and MMAs doing no work), one warpgroup spent ~0.7 us per group on it. At M = 32
+// two warpgroups save ~0.6 us per call; at MN = 48 (K=4096, N=6144) one warpgroup made the call
+// slower (44.8 us) than MN = 64 with two (34.4 us).
+__host__ __device__ constexpr int epi_warps(int mn) { return mn >= 32 ? 8 : 4; }
 // Warps: dequantisers, weight producers, an activation producer, the MMA issuer, the epilogue.
 __host__ __device__ constexpr int tc_threads(int mn) {
     return (deq_warps(mn) + wproducer_warps(mn) + 2 + epi_warps(mn)) * 32;
@@ -548,13 +548,36 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             }
             ptx::tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(C::kDCol + db * MN + m0);
-#pragma unroll
-            for (int c0 = 0; c0 < EH; c0 += 16) {
-                uint32_t v[16];
-                ptx::tmem_ld_32x32b_x16(taddr + c0, v);
+            // Loads of 16 columns start on 16-column boundaries, of 8 on 8-column ones: a half of
+            // MN = 48, 80 or 112 (24, 40 or 56 columns) reads its odd 8 columns with one x8 load,
+            // first in the upper half (which starts 8 past a 16-column boundary), last in the lower.
+            if (EH % 16 != 0 && m0 != 0) {
+                uint32_t v[8];
+                ptx::tmem_ld_32x32b_x8(taddr, v);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 16; ++q) tot[c0 + q] = fmaf(sc, __uint_as_float(v[q]), tot[c0 + q]);
+                for (int q = 0; q < 8; ++q) tot[q] = fmaf(sc, __uint_as_float(v[q]), tot[q]);
+            }
+            const int c_off = (EH % 16 != 0 && m0 != 0) ? 8 : 0;
+#pragma unroll
+            for (int c0 = 0; c0 + 16 <= EH; c0 += 16) {
+                uint32_t v[16];
+                ptx::tmem_ld_32x32b_x16(taddr + c_off + c0, v);
+                ptx::tmem_wait_ld();
+                if (c_off) {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) tot[8 + c0 + q] = fmaf(sc, __uint_as_float(v[q]), tot[8 + c0 + q]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) tot[c0 + q] = fmaf(sc, __uint_as_float(v[q]), tot[c0 + q]);
+                }
+            }
+            if (EH % 16 != 0 && m0 == 0) {
+                uint32_t v[8];
+                ptx::tmem_ld_32x32b_x8(taddr + (EH - 8), v);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 8; ++q) tot[EH - 8 + q] = fmaf(sc, __uint_as_float(v[q]), tot[EH - 8 + q]);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(ptx::smem_addr(&bar_dempty[db]));
