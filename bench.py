@@ -181,8 +181,8 @@ class Problem:
                           workspace=self.ws, stream=stream, pdl=self.pdl, out_f32=self.out_f32)
 
     def launches_per_step(self):
-        # The library's automatic choice: tensor-core GEMM (one launch per 128 rows) above 32 rows,
-        # and for 17..32 rows when N has at least 96 tiles of 128 columns; otherwise the GEMV (one
+        # The library's automatic choice: tensor-core GEMM (one launch per 128 rows) above 24 rows,
+        # and for 17..24 rows when N has at least 96 tiles of 128 columns; otherwise the GEMV (one
         # launch per 16 rows).
         return (self.M + 127) // 128 if uses_tc(self.M, self.N, self.K) else (self.M + 15) // 16
 
