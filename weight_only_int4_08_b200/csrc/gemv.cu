@@ -99,6 +99,9 @@ __device__ __forceinline__ void lds_words(const uint32_t* p, uint32_t (&w)[V]) {
     }
 }
 
+// fp32 form of the exponent-bias ("magic number") unpack (Kim et al. 2022; Frantar et al. 2024,
+// MARLIN), from the IEEE-754 layout: 0x4B000000 is 2^23, whose ulp is 1, so OR-ing an integer
+// below 2^23 into its mantissa gives exactly 2^23 + that integer.
 __device__ __forceinline__ float magic(uint32_t bits) { return __uint_as_float(bits | 0x4B000000u); }
 
 // Column pairs (0,1) (2,3) (4,5) (6,7) of one packed word as 2^23 + 2^(4(j%4)) * q_j.

@@ -164,6 +164,10 @@ __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t saddr, uint32_t& r0, 
                  : "memory");
 }
 
+// The unpack is the exponent-bias ("magic number") technique published by Kim et al. 2022 ("Who
+// Says Elephants Can't Run") and Frantar et al. 2024 ("MARLIN"), written here from the IEEE-754
+// layout: OR a nibble into the mantissa of an fp16 whose ulp is 1 (1024.0 = 0x6400) and the
+// value is exactly 1024 + q; subtracting 1024 + z leaves q - z exactly.
 constexpr uint32_t kMagic = 0x64006400u;      // fp16 1024.0 in both halves
 // Measured on B200: with both masks of (x & mask) | kMagic as compile-time constants the
 // compiler emits two logic instructions per unpacked register pair; with kMagic in a register

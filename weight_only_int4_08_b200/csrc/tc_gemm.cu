@@ -10,7 +10,9 @@
 // (q - z) is an integer in [-15, 15]: exact in fp16, and its products with the
 // fp16 activations are exact in the fp32 accumulator, so each group's partial
 // sum D_g is exact up to fp32 summation; the fp16 scale is applied in fp32 when
-// D_g is read back (tot += s[g, n] * D_g), never rounded into the weights.
+// D_g is read back (tot += s[g, n] * D_g), never rounded into the weights. The exact unpack is
+// the exponent-bias ("magic number") technique of Kim et al. 2022 and Frantar et al. 2024
+// (MARLIN), derived here from the fp16 layout: 0x6400 | q is 1024 + q.
 //
 // Roles (one CTA = one 128-column tile x one K slab; 19 warps, 15 at MN = 16):
 //   warps 0-7   dequantisers: warp p owns TMEM lanes 32(p%4)..+31 and tile
