@@ -67,12 +67,38 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_only(text):
+    """C/CUDA source with its comments removed and every run of whitespace made one space, so that
+    a change to comments or layout alone does not count as a change of the code."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":                                   # string or character literal, kept whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def csrc_hash(files=None):
-    """Hash of the library sources a kernel is compiled from (all of csrc/ when files is None)."""
+    """Hash of the code (comments and layout ignored) of the library sources a kernel is compiled
+    from (all of csrc/ when files is None)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "weight_only_int4_08_b200", "csrc")
     for f in sorted(files or os.listdir(d)):
-        h.update(open(os.path.join(d, f), "rb").read())
+        h.update(code_only(open(os.path.join(d, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -40,3 +40,13 @@ def test_cpu_baseline_takes_a_checkpoint_layout_case():
     assert c.get("b") is None
     r = bench.cpu_baseline(c, seconds=0.01)
     assert r["kind"] == "oracle" and r["value"] > 0 and "M=4 K=256 N=64" in r["sample"]
+
+
+def test_source_hash_ignores_comments_and_layout_only():
+    """The traffic record is tied to the kernel's code: comments and whitespace do not change the
+    hash, a change inside a string literal or of a token does."""
+    import bench
+    base = 'int a = 1; // one\n/* two\n lines */ const char* s = "x // y"; char c = \'"\';\n'
+    assert bench.code_only(base) == bench.code_only('int a = 1;\nconst char* s = "x // y";  char c = \'"\'; // z\n')
+    assert bench.code_only(base) != bench.code_only(base.replace('"x // y"', '"x //  y"'))
+    assert bench.code_only(base) != bench.code_only(base.replace("a = 1", "a = 2"))
