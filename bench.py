@@ -68,16 +68,23 @@ def load_peaks():
 
 
 def code_only(text):
-    """C/CUDA source with its comments removed and every run of whitespace made one space, so that
-    a change to comments or layout alone does not count as a change of the code."""
-    out, i, n = [], 0, len(text)
+    """C/CUDA source with its comments removed and every run of whitespace outside string and
+    character literals made one space, so that a change to comments or layout alone does not count
+    as a change of the code (literals, inline assembly included, are kept as written)."""
+    parts, code, i, n = [], [], 0, len(text)
+
+    def flush():
+        parts.append(" ".join("".join(code).split()))
+        code.clear()
+
     while i < n:
         c = text[i]
         if c in "\"'":                                   # string or character literal, kept whole
             j = i + 1
             while j < n and text[j] != c:
                 j += 2 if text[j] == "\\" else 1
-            out.append(text[i:j + 1])
+            flush()
+            parts.append(text[i:j + 1])
             i = j + 1
         elif text.startswith("//", i):
             j = text.find("\n", i)
@@ -85,11 +92,12 @@ def code_only(text):
         elif text.startswith("/*", i):
             j = text.find("*/", i + 2)
             i = n if j < 0 else j + 2
-            out.append(" ")
+            code.append(" ")
         else:
-            out.append(c)
+            code.append(c)
             i += 1
-    return " ".join("".join(out).split())
+    flush()
+    return " ".join(p for p in parts if p)
 
 
 def csrc_hash(files=None):
