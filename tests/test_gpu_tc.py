@@ -57,6 +57,27 @@ def test_tc_batch_layer_large_batches(w, M):
     assert_close(out[:, cols], ref(c, cols=cols), f"TC M={M}")
 
 
+def test_tc_batch_layer_256_rows_weights_from_dram(w):
+    """256 rows of the batch layer with the weights, scales and zeros starting in DRAM: a fill of
+    256 MB (twice the L2) after the operands are on the device evicts them, then one call runs its
+    two 128-row launches back to back. Every row is checked against the oracle on sampled columns.
+    Under ncu with --cache-control none this is the case that shows how many bytes a call reads
+    from DRAM (the second launch finds the layer in L2)."""
+    M, K, N = 256, 4096, 14336
+    c = synth.make_case(M, K, N, 128, sym=False, seed=4)
+    a, b, s, z = dev(c["a"]), dev(c["b"]), dev(c["s"]), dev(c["z"])
+    out = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    ws = w.alloc_workspace(M, N, K, 128, kernel=w.KERNEL_TC)
+    evict = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    evict.fill_(1)
+    w.w4a16_gemm(a, b, s, z, 128, 0, out=out, workspace=ws, kernel=w.KERNEL_TC)
+    torch.cuda.synchronize()
+    del evict
+    g = np.random.default_rng(256)
+    cols = np.unique(np.concatenate([np.arange(0, N, 128) + g.integers(0, 128, N // 128), [0, N - 1]]))
+    assert_close(out.cpu().numpy()[:, cols], ref(c, cols=cols), "TC M=256 from DRAM")
+
+
 @pytest.mark.parametrize("G", [16, 32, 64, 128, 256])
 @pytest.mark.parametrize("split", [1, 3])
 def test_tc_group_sizes_and_splits(w, G, split):
