@@ -174,8 +174,9 @@ KERNELS = {"GEMV": 1, "TC": 2, "GEMV_FMA": 3}
     (25, 6144, 4096, 128, {}, "TC"),             # above 24 rows: the GEMM whenever it can
     (24, 12288, 4096, 128, {}, "TC"),            # exactly 96
     (24, 12160, 4096, 128, {}, "GEMV"),          # 95
-    (24, 4096, 14336, 128, {}, "GEMV"),          # a long K alone does not take the GEMM
-    (28, 4096, 14336, 128, {}, "TC"),
+    (24, 4096, 14336, 128, {}, "TC"),            # K >= 8192: a long K splits into enough CTAs
+    (17, 4096, 8192, 128, {}, "TC"),
+    (24, 4096, 8064, 128, {}, "GEMV"),           # K < 8192 on a narrow layer
     (32, 4096, 8064, 128, {}, "TC"),
     (33, 4096, 4096, 128, {}, "TC"),
     (64, 4096, 4160, 64, {}, "GEMV"),            # K % 128 != 0
