@@ -215,9 +215,8 @@ class Problem:
                           workspace=self.ws, stream=stream, pdl=self.pdl, out_f32=self.out_f32)
 
     def launches_per_step(self):
-        # The library's automatic choice: tensor-core GEMM (one launch per 128 rows) above 24 rows,
-        # and for 17..24 rows when N has at least 96 tiles of 128 columns or K >= 8192; otherwise the GEMV (one
-        # launch per 16 rows).
+        # The library's automatic choice: tensor-core GEMM (one launch per 128 rows) above 16 rows,
+        # otherwise the GEMV (one launch).
         return (self.M + 127) // 128 if uses_tc(self.M, self.N, self.K) else (self.M + 15) // 16
 
 
@@ -227,7 +226,7 @@ def copies_for(bytes_per_copy):
 
 def uses_tc(M, N, K=4096):
     """The library's automatic kernel choice for an aligned problem (see w4a16_api.cu)."""
-    return M > 24 or (M > 16 and (N // 128 >= 96 or K >= 8192))
+    return M > 16
 
 
 def capture(torch, fn, n):

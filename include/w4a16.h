@@ -142,10 +142,9 @@ W4A16_API size_t w4a16_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int
  *             symmetric form, where every zero point is zp_bias. When qzeros is
  *             given, zp_bias is ignored.
  *   M, N, K   M >= 1, N >= 8, K >= group_size; N % 8 == 0; K % group_size == 0.
- *             M <= 16 runs the GEMV (warp mma.sync, one launch per 16 rows);
- *             larger M the tcgen05 tensor-core GEMM when its shape and
- *             alignment rules hold, except that 17..24 rows stay on the GEMV
- *             when N has fewer than 96 tiles of 128 columns and K < 8192.
+ *             M <= 16 runs the GEMV (warp mma.sync, one launch); larger M the
+ *             tcgen05 tensor-core GEMM when its shape and alignment rules
+ *             hold, otherwise the GEMV once per 16 rows.
  *   group_size G: G >= 16 and G % 16 == 0.
  *   zp_bias   0..15 when qzeros is NULL.
  *   out       fp16 [M, N], device, 2-byte aligned; fully overwritten; must not
@@ -172,7 +171,7 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
 /*
  * Kernel selection for tests and measurement.
  *   kernel: W4A16_KERNEL_AUTO uses the same table as w4a16_gemm (GEMV for
- *     M <= 16, and for 17..24 rows when N / 128 < 96 and K < 8192; tensor cores otherwise
+ *     M <= 16; tensor cores otherwise
  *     when N % 128 == 0, K % 128 == 0 and a, b_packed are 16-byte aligned); GEMV forces the GEMV family (any M; larger
  *     M runs it once per block of 16 rows of A): its multiply-accumulate uses
  *     warp mma.sync when N % 32 == 0, a and b_packed are 16-byte and scales

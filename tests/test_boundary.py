@@ -168,16 +168,14 @@ KERNELS = {"GEMV": 1, "TC": 2, "GEMV_FMA": 3}
 @pytest.mark.parametrize("M,N,K,G,ptrs,expect", [
     (1, 14336, 4096, 128, {}, "GEMV"),
     (16, 14336, 4096, 128, {}, "GEMV"),          # one GEMV launch
-    (17, 14336, 4096, 128, {}, "TC"),            # 112 column tiles >= 96
+    (17, 14336, 4096, 128, {}, "TC"),            # above 16 rows: the GEMM whenever it can
     (32, 14336, 4096, 128, {}, "TC"),
-    (24, 6144, 4096, 128, {}, "GEMV"),           # 48 column tiles
-    (25, 6144, 4096, 128, {}, "TC"),             # above 24 rows: the GEMM whenever it can
-    (24, 12288, 4096, 128, {}, "TC"),            # exactly 96
-    (24, 12160, 4096, 128, {}, "GEMV"),          # 95
-    (24, 4096, 14336, 128, {}, "TC"),            # K >= 8192: a long K splits into enough CTAs
-    (17, 4096, 8192, 128, {}, "TC"),
-    (24, 4096, 8064, 128, {}, "GEMV"),           # K < 8192 on a narrow layer
-    (32, 4096, 8064, 128, {}, "TC"),
+    (16, 6144, 4096, 128, {}, "GEMV"),           # one GEMV launch
+    (17, 6144, 4096, 128, {}, "TC"),
+    (17, 4096, 4096, 128, {}, "TC"),
+    (24, 4096, 14336, 128, {}, "TC"),
+    (17, 4096, 8064, 128, {}, "TC"),             # 8064 = 63 x 128
+    (16, 4096, 14336, 128, {}, "GEMV"),
     (33, 4096, 4096, 128, {}, "TC"),
     (64, 4096, 4160, 64, {}, "GEMV"),            # K % 128 != 0
     (64, 4128, 4096, 128, {}, "GEMV"),           # N % 128 != 0, N % 32 == 0

@@ -82,22 +82,21 @@ struct Choice {
 };
 
 // Kernel table. M <= 16: the mma.sync GEMV (one launch; the CUDA-core GEMV when its
-// alignment rules fail). 17..24 rows: the GEMV needs two launches, each reading all the
-// weights, while the tensor-core GEMM reads them once, one CTA per 128 columns (times a K
-// split); the GEMM is taken when N has at least 96 such column tiles, or when K is at least
-// 8192 (a long K splits into enough CTAs to fill the GPU). Above 24 rows: the GEMM. The GEMM
-// only when the shape and pointers allow it (N % 128, K % 128, 16-byte aligned A and weights),
-// the GEMV's row blocks otherwise. Null pointers (workspace query) count as aligned.
-// Measured on B200, G=128, CUDA graphs with programmatic dependent launch, weights larger than
-// L2 (GEMV / GEMM, us):
-//   K=4096 N=6144:   M=17 18.8 / 20.7, M=24 20.6 / 21.2, M=28 23.0 / 21.2, M=40 32.2 / 28.4
-//   K=4096 N=4096:   M=17 14.5 / 16.4, M=24 15.9 / 16.7, M=28 17.6 / 17.0, M=40 24.8 / 21.9
-//   K=14336 N=4096:  M=17 27.7 / 25.3, M=20 28.6 / 26.0, M=32 33.2 / 26.4
-//   K=4096 N=28672:  M=17 61.3 / 36.4, M=20 69.9 / 36.3, M=32 63.5 / 36.4
-//   K=4096 N=14336:  M=17 25.5 / 18.3, M=24 27.6 / 18.1
-constexpr int64_t kGemvOneLaunchM = 16, kGemvMaxM = 24, kTcMinTiles = 96, kTcMinK = 8192;
+// alignment rules fail). Above 16 rows the GEMV needs a second launch that reads all the weights
+// again, while the tensor-core GEMM reads them once: the GEMM, whenever the shape and pointers
+// allow it (N % 128, K % 128, 16-byte aligned A and weights), the GEMV's row blocks otherwise.
+// Null pointers (workspace query) count as aligned. Measured on B200, G=128, CUDA graphs with
+// programmatic dependent launch, weights larger than L2 (GEMV / GEMM, us):
+//   K=4096 N=6144:   M=16 11.9 / 12.5, M=17 18.8 / 13.2, M=24 20.7 / 13.4
+//   K=4096 N=4096:   M=16  9.2 / 11.3, M=17 14.5 / 11.6, M=24 16.0 / 11.9
+//   K=14336 N=4096:  M=16 16.7 / 19.7, M=17 27.6 / 20.8, M=24 29.8 / 20.9
+//   K=4096 N=14336:  M=16 15.9 / 17.4, M=17 25.5 / 18.1, M=24 27.5 / 18.0
+//   K=4096 N=28672:  M=17 61.3 / 36.4, M=32 63.5 / 36.4
+constexpr int64_t kGemvOneLaunchM = 16;
 bool auto_prefers_tc(int64_t M, int64_t N, int64_t K) {
-    return M > kGemvMaxM || (M > kGemvOneLaunchM && (N / 128 >= kTcMinTiles || K >= kTcMinK));
+    (void)N;
+    (void)K;
+    return M > kGemvOneLaunchM;
 }
 Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms,
               const void* a, const void* b, const void* s, const void* z) {
