@@ -159,11 +159,7 @@ struct SegIter {
 };
 
 // FAST: G is a multiple of the stage (kStageK rows), so group segments are whole stages.
-// SPLIT: the K range is split between CTAs (p.split > 1), whose fp32 partials the last-arriving
-// CTA of each tile adds up; launches without a split are compiled without that code, which would
-// otherwise take registers from the main loops (measured on B200: M=32, K=4096, N=14336,
-// 18.63 -> 18.80 us with it).
-template <int MN, bool FAST, bool SPLIT>
+template <int MN, bool FAST>
 __global__ void __launch_bounds__(tc_threads(MN), 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap, TcArgs p) {
     using C = TcCfg<MN>;
@@ -597,7 +593,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const bool bad = ptx::named_bar_or(1, kEpiThreads, !ok || s_abort);
         asm volatile("griddepcontrol.wait;" ::: "memory");   // before the first write
         if (!bad) {
-            if constexpr (!SPLIT) {
+            if (p.split == 1) {
                 // The tile goes out through shared memory: every stage has been consumed (the last
                 // group's accumulator is complete, so every MMA, and before them every dequantiser
                 // read and every load, has finished), so the weight ring is idle. Each thread puts its
@@ -642,23 +638,33 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 if (s_last) {
                     // The last-arriving CTA adds the tile's partials in split order (0 + p0 + p1 + ...).
                     __threadfence();
-                    // The partials of one split for a block of 8 rows are loaded together, and the
-                    // block is stored after the last split. Measured on B200 (K=N=4096, M=32, split
-                    // 4): a row-by-row loop, whose store kept the next row's loads waiting, took
-                    // ~11 us in these CTAs against ~2 us for the others; the call 19.4 -> 13.7 us.
+                    if constexpr (EH <= 32) {
+                        // The partials of one split for a block of 8 rows are loaded together, and
+                        // the block is stored after the last split. Measured on B200 (K=N=4096,
+                        // M=32, split 4): the row-by-row loop below, whose store keeps the next
+                        // row's loads waiting, took ~11 us in these CTAs against ~2 us for the
+                        // others; the call 19.4 -> 13.7 us. (Above 32 rows per warpgroup the blocks
+                        // cost the kernel's main loops registers: M=128 26.8 -> 29.8 us unsplit.)
 #pragma unroll
-                    for (int c0 = 0; c0 < EH; c0 += 8) {
+                        for (int c0 = 0; c0 < EH; c0 += 8) {
 #pragma unroll
-                        for (int m = c0; m < c0 + 8 && m < EH; ++m) tot[m] = 0.f;
-                        for (int y = 0; y < p.split; ++y) {
-                            const float* py = p.partials + ((int64_t)y * p.mblk + m0) * p.N + n;
+                            for (int m = c0; m < c0 + 8 && m < EH; ++m) tot[m] = 0.f;
+                            for (int y = 0; y < p.split; ++y) {
+                                const float* py = p.partials + ((int64_t)y * p.mblk + m0) * p.N + n;
+#pragma unroll
+                                for (int m = c0; m < c0 + 8 && m < EH; ++m)
+                                    if (m0 + m < p.mblk) tot[m] += __ldcg(py + (int64_t)m * p.N);
+                            }
 #pragma unroll
                             for (int m = c0; m < c0 + 8 && m < EH; ++m)
-                                if (m0 + m < p.mblk) tot[m] += __ldcg(py + (int64_t)m * p.N);
+                                if (m0 + m < p.mblk) p.out.put((int64_t)(m0 + m) * p.N + n, tot[m]);
                         }
-#pragma unroll
-                        for (int m = c0; m < c0 + 8 && m < EH; ++m)
-                            if (m0 + m < p.mblk) p.out.put((int64_t)(m0 + m) * p.N + n, tot[m]);
+                    } else {
+                        for (int m = m0; m < min(m0 + EH, p.mblk); ++m) {
+                            float a = 0.f;
+                            for (int y = 0; y < p.split; ++y) a += __ldcg(p.partials + ((int64_t)y * p.mblk + m) * p.N + n);
+                            p.out.put((int64_t)m * p.N + n, a);
+                        }
                     }
                     if (et == 0) p.counters[tile] = 0u;
                 }
@@ -680,23 +686,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 
 using TcFn = void (*)(CUtensorMap, CUtensorMap, TcArgs);
 
-template <bool FAST, bool SPLIT>
+template <bool FAST>
 TcFn select_tc_t(int mn) {
     switch (mn) {
-        case 16: return tc_gemm_kernel<16, FAST, SPLIT>;
-        case 32: return tc_gemm_kernel<32, FAST, SPLIT>;
-        case 48: return tc_gemm_kernel<48, FAST, SPLIT>;
-        case 64: return tc_gemm_kernel<64, FAST, SPLIT>;
-        case 80: return tc_gemm_kernel<80, FAST, SPLIT>;
-        case 96: return tc_gemm_kernel<96, FAST, SPLIT>;
-        case 112: return tc_gemm_kernel<112, FAST, SPLIT>;
-        default: return tc_gemm_kernel<128, FAST, SPLIT>;
+        case 16: return tc_gemm_kernel<16, FAST>;
+        case 32: return tc_gemm_kernel<32, FAST>;
+        case 48: return tc_gemm_kernel<48, FAST>;
+        case 64: return tc_gemm_kernel<64, FAST>;
+        case 80: return tc_gemm_kernel<80, FAST>;
+        case 96: return tc_gemm_kernel<96, FAST>;
+        case 112: return tc_gemm_kernel<112, FAST>;
+        default: return tc_gemm_kernel<128, FAST>;
     }
 }
-TcFn select_tc(int mn, bool fast, bool split) {
-    return fast ? (split ? select_tc_t<true, true>(mn) : select_tc_t<true, false>(mn))
-                : (split ? select_tc_t<false, true>(mn) : select_tc_t<false, false>(mn));
-}
+TcFn select_tc(int mn, bool fast) { return fast ? select_tc_t<true>(mn) : select_tc_t<false>(mn); }
 
 size_t tc_smem(int mn) {
     switch (mn) {
@@ -725,7 +728,7 @@ int tc_ctas_per_sm(int mn) {
     // Resident CTAs per SM from the three budgets the kernel draws on: shared
     // memory (228 KB per SM, 1 KB reserved per CTA), registers (64 K per SM)
     // and tensor memory (512 columns per SM).
-    TcFn k = select_tc(mn, true, true);   // the split form: the more registers of the two
+    TcFn k = select_tc(mn, true);
     const size_t smem = tc_launch_smem(mn);
     cudaFuncAttributes fa{};
     int regs = 255;
@@ -825,7 +828,7 @@ cudaError_t launch_tc(const __half* a, const uint32_t* b, const __half* s, const
         args.wait_ns = wp.limit_ns;
         // Every row block uses the plan's MN (the largest); a short last block
         // leaves its padded rows to TMA's zero fill.
-        TcFn k = select_tc(pl.mn, G % kStageK == 0, pl.split_k > 1);
+        TcFn k = select_tc(pl.mn, G % kStageK == 0);
         const size_t smem = tc_launch_smem(pl.mn);
         e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
