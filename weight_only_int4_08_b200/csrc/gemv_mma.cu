@@ -335,6 +335,27 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
 #pragma unroll
         for (int j = 0; j < kRing; ++j) first_kb[j] = arm_w();
     }
+    // Copy group gg's scales and zero words of a tile into group buffer gg & 1 (lane l copies scales
+    // 4l..4l+3, lanes 0..15 the zero words), one group ahead of use. Chunks past N get zero scales.
+    auto load_meta = [&](int tile, int gg) {
+        unsigned char* gb = grp + (gg & 1) * kGrpBytes;
+        if ((int64_t)tile * kTileN + 32 * (lane / 8) < p.N)
+            cp_async_8(ptx::smem_addr(gb + 8 * lane), p.s + (int64_t)tile * kTileN + 4 * lane + (int64_t)gg * p.N);
+        else
+            *reinterpret_cast<uint2*>(gb + 8 * lane) = make_uint2(0u, 0u);
+        if (p.z && lane < kTileWords && tile * kTileWords + lane < nw)
+            cp_async_4(ptx::smem_addr(gb + 2 * kTileN + 4 * lane), p.z + (int64_t)tile * kTileWords + lane + (int64_t)gg * nw);
+        cp_async_commit();
+    };
+    // The first fragment's first group goes out before the wait for the previous kernel: like the
+    // weights, scales and zeros are written by no kernel this one may overlap. Measured on B200
+    // (per-warp timeline, K=N=4096, M=1, one 8 KB unit per warp): the first group's copy issued
+    // after the wait held the warp ~0.3 us once its weights had landed.
+    if (nfrag > 0) {
+        int lo0, hi0;
+        frag_lo_hi(0, lo0, hi0);
+        if (lo0 < hi0) load_meta(t0, lo0 * kRows / G);
+    }
     __syncthreads();   // the abort flag and the zero row are set
     if (cluster_shares) cluster_arrive_relaxed();
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -382,11 +403,6 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         int lo, hi;
         frag_lo_hi(f, lo, hi);
         const int rend = min(hi * kRows, K);
-        // This tile's group-0 scale row (lane l copies scales 4l..4l+3) and zero row (lanes 0..15).
-        const __half* s_tile = p.s + (int64_t)tile * kTileN + 4 * lane;
-        const uint32_t* z_tile = p.z ? p.z + (int64_t)tile * kTileWords + lane : nullptr;
-        const bool s_ok = (int64_t)tile * kTileN + 32 * (lane / 8) < p.N;
-        const bool z_ok = p.z && lane < kTileWords && tile * kTileWords + lane < nw;
 
         float acc[4][NT][8];
         // The fragment's scaled group sums: in registers up to 8 rows (4 NI values per lane, stored to
@@ -401,17 +417,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             else tmine[32 * k] = 0.f;
         }
 
-        // Copy group gg's scales and zero words of this tile into group buffer gg & 1, one group
-        // ahead of use. Chunks past N get zero scales.
-        auto load_group = [&](int gg) {
-            unsigned char* gb = grp + (gg & 1) * kGrpBytes;
-            if (s_ok)
-                cp_async_8(ptx::smem_addr(gb + 8 * lane), s_tile + (int64_t)gg * p.N);
-            else
-                *reinterpret_cast<uint2*>(gb + 8 * lane) = make_uint2(0u, 0u);
-            if (z_ok) cp_async_4(ptx::smem_addr(gb + 2 * kTileN + 4 * lane), z_tile + (int64_t)gg * nw);
-            cp_async_commit();
-        };
+        auto load_group = [&](int gg) { load_meta(tile, gg); };
         // Groups advance one at a time: g_cur is the open group (from g_first), g_next its end row.
         const int g_first = lo * kRows / G;
         int g_cur = g_first - 1, g_next = g_first * G;
@@ -486,7 +492,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
             }
         };
 
-        if (lo < hi) load_group(g_first);
+        if (lo < hi && f > 0) load_group(g_first);   // (fragment 0's went out before the wait)
         for (int kb = lo; kb < hi && !failed; ++kb) {
             const int slot = consumed % kRing;
             const bool okw = ptx::mbar_wait(bar0 + 8 * slot, (uint32_t)((consumed / kRing) & 1), &s_abort, p.wait_ns);
