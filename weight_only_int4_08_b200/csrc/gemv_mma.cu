@@ -29,13 +29,15 @@
 // TMA boxes of 64 B x 16..32 rows ran up to 2x slower than boxes of 4 KB and
 // more, and about 128 KB in flight per SM was enough; and one resident CTA per
 // SM with 128-row stages needs fewer instructions per byte (no register cap,
-// half the per-stage bookkeeping) than two CTAs with 64-row stages. Scales and zero words are copied one group ahead into a small
-// per-warp shared buffer (cp.async); each group's scaled sums are added to
-// fp32 totals kept in shared memory. At the end of a fragment the warps are
-// reduced in warp order; a tile covered by one CTA is
-// written directly, otherwise each CTA stores its fp32 partial in a slot of its
-// own and the last-arriving CTA sums the slots in CTA order (fixed order, no
-// floating-point atomics: bit-reproducible).
+// half the per-stage bookkeeping) than two CTAs with 64-row stages. Scales and
+// zero words are copied one group ahead into a small per-warp shared buffer
+// (cp.async; the first group before the wait on the previous kernel); each
+// group's scaled sums are added to fp32 totals kept in registers. At the end of
+// a fragment the totals go to shared memory and the warps are reduced in warp
+// order; a tile covered by one CTA is written directly, otherwise the CTAs of
+// the thread-block cluster that share it store their parts into the first one's
+// shared memory, which adds them in rank order after one cluster barrier (fixed
+// order, no floating-point atomics: bit-reproducible).
 //
 // Register layout (lane = 4 g + t): ldmatrix.trans gives thread (g, t) the
 // k-pair t of an 8-row matrix for columns 4g..4g+3 of a 32-column chunk; MMA 1
@@ -405,17 +407,14 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         const int rend = min(hi * kRows, K);
 
         float acc[4][NT][8];
-        // The fragment's scaled group sums: in registers up to 8 rows (4 NI values per lane, stored to
-        // shared memory once at the fragment's end), in shared memory above, where registers run out.
-        // Measured on B200 (decode GEMV, per-warp timeline): 16 load-FMA-store steps on shared memory
-        // took ~0.24 us per group.
-        constexpr bool kRegTot = MT <= 8;
-        float treg[kRegTot ? 4 * NI : 1];
+        // The fragment's scaled group sums, in registers (4 NI values per lane, stored to shared
+        // memory once at the fragment's end). Measured on B200: at one row (per-warp timeline) the
+        // 16 load-FMA-store steps on shared memory they replaced took ~0.24 us per group; at 9-16
+        // rows (64 per group, the kernel at 234-237 registers without spills) they cost 4-10 %, e.g.
+        // K=4096, N=14336, M=16 16.2 -> 14.7 us.
+        float treg[4 * NI];
 #pragma unroll
-        for (int k = 0; k < 4 * NI; ++k) {
-            if constexpr (kRegTot) treg[k] = 0.f;
-            else tmine[32 * k] = 0.f;
-        }
+        for (int k = 0; k < 4 * NI; ++k) treg[k] = 0.f;
 
         auto load_group = [&](int gg) { load_meta(tile, gg); };
         // Groups advance one at a time: g_cur is the open group (from g_first), g_next its end row.
@@ -435,12 +434,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
                     for (int i = 0; i < 8; ++i)
                         if (MT > 1 || (i & 1) == 0) {
                             const int k = c * NI + nt * NB + (MT > 1 ? i : i / 2);
-                            if constexpr (kRegTot) {
-                                treg[k] = fmaf(sj[i >> 1], acc[c][nt][i], treg[k]);
-                            } else {
-                                float* tp = tmine + 32 * k;
-                                *tp = fmaf(sj[i >> 1], acc[c][nt][i], *tp);
-                            }
+                            treg[k] = fmaf(sj[i >> 1], acc[c][nt][i], treg[k]);
                         }
             }
         };
@@ -556,10 +550,8 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__
         // ---- reduce fragment f over the warps (warp order) ----
         // A tile held by this CTA alone is written out now; the first and the last fragment may be
         // shared with other CTAs of the cluster and are kept (keep[0], keep[1]) for the exchange.
-        if constexpr (kRegTot) {
 #pragma unroll
-            for (int k = 0; k < 4 * NI; ++k) tmine[32 * k] = treg[k];
-        }
+        for (int k = 0; k < 4 * NI; ++k) tmine[32 * k] = treg[k];
         __syncthreads();
         // s_abort is read by every thread between two barriers with no wait in between: uniform.
         if (s_abort == 0) {
