@@ -87,10 +87,10 @@ struct Choice {
 // allow it (N % 128, K % 128, 16-byte aligned A and weights), the GEMV's row blocks otherwise.
 // Null pointers (workspace query) count as aligned. Measured on B200, G=128, CUDA graphs with
 // programmatic dependent launch, weights larger than L2 (GEMV / GEMM, us):
-//   K=4096 N=6144:   M=16 11.9 / 12.5, M=17 18.8 / 13.2, M=24 20.7 / 13.4
+//   K=4096 N=6144:   M=16 11.1 / 12.5, M=17 18.8 / 13.2, M=24 20.7 / 13.4
 //   K=4096 N=4096:   M=16  9.2 / 11.3, M=17 14.5 / 11.6, M=24 16.0 / 11.9
-//   K=14336 N=4096:  M=16 16.7 / 19.7, M=17 27.6 / 20.8, M=24 29.8 / 20.9
-//   K=4096 N=14336:  M=16 15.9 / 17.4, M=17 25.5 / 18.1, M=24 27.5 / 18.0
+//   K=14336 N=4096:  M=16 15.7 / 19.7, M=17 27.6 / 20.8, M=24 29.8 / 20.9
+//   K=4096 N=14336:  M=16 14.7 / 17.4, M=17 25.5 / 18.1, M=24 27.5 / 18.0
 //   K=4096 N=28672:  M=17 61.3 / 36.4, M=32 63.5 / 36.4
 constexpr int64_t kGemvOneLaunchM = 16;
 bool auto_prefers_tc(int64_t M, int64_t N, int64_t K) {
