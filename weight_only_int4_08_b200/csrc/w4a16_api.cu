@@ -91,7 +91,7 @@ struct Choice {
 //   K=4096 N=4096:   M=16  9.2 / 11.3, M=17 14.5 / 11.6, M=24 16.0 / 11.9
 //   K=14336 N=4096:  M=16 15.7 / 19.7, M=17 27.6 / 20.8, M=24 29.8 / 20.9
 //   K=4096 N=14336:  M=16 14.7 / 17.4, M=17 25.5 / 18.1, M=24 27.5 / 18.0
-//   K=4096 N=28672:  M=17 61.3 / 36.4, M=32 63.5 / 36.4
+//   K=4096 N=28672:  M=16 30.9 / 34.8, M=17 61.3 / 36.4, M=32 63.5 / 36.4
 constexpr int64_t kGemvOneLaunchM = 16;
 bool auto_prefers_tc(int64_t M, int64_t N, int64_t K) {
     (void)N;
