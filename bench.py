@@ -225,7 +225,8 @@ def copies_for(bytes_per_copy):
 
 
 def uses_tc(M, N, K=4096):
-    """The library's automatic kernel choice for an aligned problem (see w4a16_api.cu)."""
+    """The library's automatic kernel choice for an aligned problem (see w4a16_api.cu): the
+    tensor-core GEMM above 16 rows, for any N and K that meet its shape rules."""
     return M > 16
 
 

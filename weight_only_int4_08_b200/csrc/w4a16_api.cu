@@ -93,11 +93,7 @@ struct Choice {
 //   K=4096 N=14336:  M=16 14.7 / 17.4, M=17 25.5 / 18.1, M=24 27.5 / 18.0
 //   K=4096 N=28672:  M=16 30.9 / 34.8, M=17 61.3 / 36.4, M=32 63.5 / 36.4
 constexpr int64_t kGemvOneLaunchM = 16;
-bool auto_prefers_tc(int64_t M, int64_t N, int64_t K) {
-    (void)N;
-    (void)K;
-    return M > kGemvOneLaunchM;
-}
+bool auto_prefers_tc(int64_t M) { return M > kGemvOneLaunchM; }
 Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_options* opts, int sms,
               const void* a, const void* b, const void* s, const void* z) {
     Choice c{};
@@ -105,7 +101,7 @@ Choice choose(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_optio
     const bool tc_ok = tc_supported(M, N, K, G, a ? a : (const void*)16, b ? b : (const void*)16);
     if (req == W4A16_KERNEL_TC) c.kernel = W4A16_KERNEL_TC;
     else if (req == W4A16_KERNEL_GEMV || req == W4A16_KERNEL_GEMV_FMA) c.kernel = W4A16_KERNEL_GEMV;
-    else c.kernel = (auto_prefers_tc(M, N, K) && tc_ok) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
+    else c.kernel = (auto_prefers_tc(M) && tc_ok) ? W4A16_KERNEL_TC : W4A16_KERNEL_GEMV;
     const int split = opts ? opts->split_k : 0;
     if (c.kernel == W4A16_KERNEL_TC) {
         if (tc_ok) c.tc = plan_tc(M, N, K, G, sms, split);
@@ -130,7 +126,7 @@ size_t ws_bound(int64_t M, int64_t N, int64_t K, int32_t G, const w4a16_gemm_opt
         if (req != W4A16_KERNEL_GEMV_FMA && N % 32 == 0) ws = std::max(ws, plan_gemv_mma(M, N, K, G, split, sms).ws_bytes);
     }
     const bool tc_shape = tc_supported(M, N, K, G, (const void*)16, (const void*)16);
-    if (tc_shape && (req == W4A16_KERNEL_TC || (req == W4A16_KERNEL_AUTO && auto_prefers_tc(M, N, K))))
+    if (tc_shape && (req == W4A16_KERNEL_TC || (req == W4A16_KERNEL_AUTO && auto_prefers_tc(M))))
         ws = std::max(ws, plan_tc(M, N, K, G, sms, opts ? opts->split_k : 0).ws_bytes);
     return ws;
 }
@@ -261,7 +257,7 @@ w4a16_status w4a16_gemm_kernel_choice(int64_t M, int64_t N, int64_t K, int32_t g
     const void* pb = b_packed ? b_packed : (const void*)16;
     const void* ps = scales ? scales : (const void*)16;
     // the same decisions as choose() and the launch path, without the device queries
-    if (auto_prefers_tc(M, N, K) && tc_supported(M, N, K, group_size, pa, pb))
+    if (auto_prefers_tc(M) && tc_supported(M, N, K, group_size, pa, pb))
         *kernel = W4A16_KERNEL_TC;
     else
         *kernel = gemv_mma_supported(N, K, pa, pb, ps, nullptr) ? W4A16_KERNEL_GEMV : W4A16_KERNEL_GEMV_FMA;
