@@ -182,6 +182,9 @@ W4A16_API w4a16_status w4a16_gemm(const void* a, const void* b_packed, const voi
  *   split_k: 0 = automatic, else (1..1024) the number of K slices the kernel
  *     splits its work into: the tensor-core GEMM clamps it to K/128, the
  *     mma.sync GEMV to a thread-block cluster (at most 4 CTAs per column tile).
+ *     The tensor-core GEMM's automatic split is one whose CTAs are all
+ *     resident at once (none when the layer has as many 128-column tiles as
+ *     the GPU has CTA slots); a requested split may take several waves.
  *   debug_flags: 0 in normal use. W4A16_DEBUG_STALL_LOADS makes the kernels'
  *     load issuers issue nothing, so every device-side wait runs out: the call
  *     then leaves W4A16_ERR_TIMEOUT in the workspace status word (read it with
