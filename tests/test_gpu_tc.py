@@ -78,18 +78,24 @@ def test_tc_batch_layer_256_rows_weights_from_dram(w):
     assert_close(out.cpu().numpy()[:, cols], ref(c, cols=cols), "TC M=256 from DRAM")
 
 
-@pytest.mark.parametrize("M,N,K,split", [
-    (17, 28672, 4096, False),   # 224 column tiles: more than one wave already, no split
-    (24, 28672, 4096, False),
-    (32, 14336, 4096, False),   # 112 tiles: a split would need a second wave
-    (32, 4096, 14336, True),    # 32 tiles: a split that stays within one wave
+@pytest.mark.parametrize("M,N,K", [
+    (17, 28672, 4096),    # 224 column tiles: more than one wave already on 148 SMs, no split
+    (24, 28672, 4096),
+    (32, 14336, 4096),    # 112 tiles: a split would need a second wave on 148 SMs
+    (32, 4096, 14336),    # 32 tiles and a long K: a split that stays within one wave
 ])
-def test_tc_automatic_split_stays_within_one_wave(w, M, N, K, split):
-    """The automatic K split of the tensor-core GEMM is one whose CTAs are all resident at once:
-    its workspace holds fp32 partials only when the layer has few enough column tiles."""
+def test_tc_automatic_split_stays_within_one_wave(w, M, N, K):
+    """The automatic K split of the tensor-core GEMM is one whose CTAs are all resident at once
+    (one CTA per SM at these row counts): its workspace holds fp32 partials only when two CTAs
+    per column tile fit on the GPU, and then for a split that fits."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    tiles = N // 128
     ws = w.w4a16_gemm_workspace_bytes(M, N, K, 128, kernel=w.KERNEL_TC)
-    partials = 2 * M * N * 4   # the smallest split's partials
-    assert (ws >= partials) == split, (M, N, K, ws)
+    split = ws // (M * N * 4)   # the partials hold split x M x N fp32 values (plus a small header)
+    if 2 * tiles > sms:
+        assert split == 0, (M, N, K, ws)
+    else:
+        assert 2 <= split and split * tiles <= sms, (M, N, K, ws, split)
 
 
 @pytest.mark.parametrize("G", [16, 32, 64, 128, 256])
